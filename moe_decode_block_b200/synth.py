@@ -1,0 +1,143 @@
+"""Seeded synthetic inputs for the MoE decode block.
+
+This module only draws random numbers; it holds none of the block's
+arithmetic.  The tests, the smoke check and the benchmark all take their
+inputs from here, so the CUDA path and the fp64 oracle always see the same
+tensors.
+
+Distributions: weights ~ N(0, 0.02) and activations ~ N(0, 1), both rounded
+once (round-to-nearest-even) from float32 to bf16.  Every tensor (and every
+expert, and every row of x) draws from its own generator whose seed is a hash
+of (seed, tensor name, index), so any subset can be regenerated on its own.
+"""
+from __future__ import annotations
+
+import dataclasses
+import hashlib
+import math
+from typing import Dict, Optional, Sequence
+
+import torch
+
+WEIGHT_STD = 0.02
+ZIPF_S = 1.2
+
+
+@dataclasses.dataclass(frozen=True)
+class BlockShape:
+    hidden: int
+    n_experts: int
+    top_k: int
+    inter: int
+    shared_inter: int
+    n_shared: int = 1
+
+    def expert_bytes(self) -> int:
+        """bf16 bytes of one routed expert (w13 + w2)."""
+        return 2 * (self.hidden * 2 * self.inter + self.inter * self.hidden)
+
+    def shared_bytes(self) -> int:
+        return self.n_shared * 2 * (self.hidden * 2 * self.shared_inter + self.shared_inter * self.hidden)
+
+    def router_bytes(self) -> int:
+        return 2 * self.hidden * self.n_experts
+
+
+TINY = BlockShape(hidden=256, n_experts=16, top_k=2, inter=128, shared_inter=128)
+FULL = BlockShape(hidden=7168, n_experts=384, top_k=8, inter=2048, shared_inter=2048)
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    shape: BlockShape
+    batch: int
+    routing: str  # "uniform" (router weights only) or "zipf" (log-prior bias added)
+    description: str
+
+
+WORKLOADS: Dict[str, Workload] = {
+    "tiny_b1": Workload("tiny_b1", TINY, 1, "uniform",
+                        "tiny block: hidden 256, 16 experts top-2, inter 128, 1 shared (inter 128), batch 1"),
+    "full_b1": Workload("full_b1", FULL, 1, "uniform",
+                        "full-size block: hidden 7168, 384 experts top-8, inter 2048, 1 shared (inter 2048), batch 1"),
+    "full_b8": Workload("full_b8", FULL, 8, "uniform", "full-size block, batch 8, uniform-ish routing"),
+    "full_b64": Workload("full_b64", FULL, 64, "uniform", "full-size block, batch 64, uniform-ish routing"),
+    "zipf_b32": Workload("zipf_b32", FULL, 32, "zipf",
+                         "full-size block, batch 32, Zipf(1.2) per-expert log-prior added to router logits"),
+}
+
+
+def seed_for(seed: int, name: str, index: int = 0) -> int:
+    """Deterministic 63-bit sub-seed for (seed, tensor name, index)."""
+    h = hashlib.blake2b(f"{seed}/{name}/{index}".encode(), digest_size=8).digest()
+    return int.from_bytes(h, "little") & ((1 << 63) - 1)
+
+
+def _normal_bf16(shape: Sequence[int], std: float, seed: int, device) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    t = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    return t.to(torch.bfloat16)
+
+
+def make_x(batch: int, hidden: int, seed: int = 0, device="cpu",
+           attempts: Optional[Sequence[int]] = None) -> torch.Tensor:
+    """Activations x [batch, hidden] bf16 ~ N(0,1).  Row b is drawn from
+    sub-seed (seed, "x", b, attempts[b]); a caller that rejects a row redraws it
+    by raising its attempt counter."""
+    rows = []
+    for b in range(batch):
+        a = 0 if attempts is None else int(attempts[b])
+        rows.append(_normal_bf16((hidden,), 1.0, seed_for(seed, f"x/{a}", b), device))
+    if not rows:
+        return torch.zeros(0, hidden, dtype=torch.bfloat16, device=device)
+    return torch.stack(rows)
+
+
+@dataclasses.dataclass
+class BlockWeights:
+    router_w: torch.Tensor          # [H, E]
+    w13: torch.Tensor               # [E, H, 2I] (expert e at w13[e])
+    w2: torch.Tensor                # [E, I, H]
+    shared_w13: Optional[torch.Tensor]  # [H, 2Is]
+    shared_w2: Optional[torch.Tensor]   # [Is, H]
+    router_bias: Optional[torch.Tensor]  # [E] float32 or None
+
+
+def make_weights(shape: BlockShape, seed: int = 0, device="cpu", routing: str = "uniform") -> BlockWeights:
+    """All weights of one block, bf16 ~ N(0, 0.02), each expert from its own
+    sub-seed.  ``routing == "zipf"`` adds the Zipf log-prior bias."""
+    H, E, I, Is = shape.hidden, shape.n_experts, shape.inter, shape.shared_inter
+    router_w = _normal_bf16((H, E), WEIGHT_STD, seed_for(seed, "router_w"), device)
+    w13 = torch.empty(E, H, 2 * I, dtype=torch.bfloat16, device=device)
+    w2 = torch.empty(E, I, H, dtype=torch.bfloat16, device=device)
+    for e in range(E):
+        w13[e] = _normal_bf16((H, 2 * I), WEIGHT_STD, seed_for(seed, "w13", e), device)
+        w2[e] = _normal_bf16((I, H), WEIGHT_STD, seed_for(seed, "w2", e), device)
+    sw13 = sw2 = None
+    if shape.n_shared:
+        sw13 = _normal_bf16((H, 2 * Is), WEIGHT_STD, seed_for(seed, "shared_w13"), device)
+        sw2 = _normal_bf16((Is, H), WEIGHT_STD, seed_for(seed, "shared_w2"), device)
+    bias = zipf_log_prior(E, seed, device) if routing == "zipf" else None
+    return BlockWeights(router_w, w13, w2, sw13, sw2, bias)
+
+
+def zipf_log_prior(n_experts: int, seed: int = 0, device="cpu", s: float = ZIPF_S) -> torch.Tensor:
+    """Per-expert bias log(q_rank(e)), q_r = r^-s / sum_r' r'^-s, with the ranks
+    assigned to experts by a seeded random permutation (so the heavy experts
+    are not simply the lowest ids).  float32 [E]."""
+    z = sum(r ** -s for r in range(1, n_experts + 1))
+    logq = [math.log((r ** -s) / z) for r in range(1, n_experts + 1)]
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed_for(seed, "zipf_perm"))
+    perm = torch.randperm(n_experts, generator=g)  # expert e gets rank perm[e] + 1
+    bias = torch.tensor([logq[int(perm[e])] for e in range(n_experts)], dtype=torch.float32)
+    return bias.to(device)
+
+
+def bf16_bits(t: torch.Tensor):
+    """numpy uint16 view of a bf16 tensor's bit patterns (copied to host)."""
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")

@@ -1,0 +1,146 @@
+"""fp64 CPU oracle of the MoE decode block -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never uses it and
+shares no code with it.
+
+Two independent implementations of the same definition:
+
+* ``moe_oracle.c`` (plain C loops, fp64, OpenMP), loaded through ctypes here;
+* ``moe_oracle_np.py`` (numpy fp64 restatement, small shapes).
+
+All array arguments are numpy arrays of bf16 *bit patterns* (``uint16``),
+row-major: x [B,H], router_w [H,E], w13[e] [H,2I], w2[e] [I,H],
+sw13 [H,2Is], sw2 [Is,H]; the optional bias is float32 [E].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+from . import moe_oracle_np as np_oracle  # noqa: F401  (re-export)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_ERRORS = {-1: "bad argument", -2: "a selected expert has no weights", -3: "out of memory"}
+
+
+def build_c_oracle(force: bool = False) -> str:
+    """Compile moe_oracle.c into oracle/liboracle.so with gcc (-O2 -fopenmp)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", "-Wall", "-o", tmp, _SRC, "-lm"]
+        )
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build_c_oracle()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.oracle_router.argtypes = [P, P, P, I, I, I, I, P, P, P]
+        lib.oracle_router.restype = I
+        lib.oracle_block.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        lib.oracle_block.restype = I
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = I
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected uint16 bf16 bit patterns, got {a.dtype}")
+    return a
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"{what}: oracle error {rc} ({_ERRORS.get(rc, 'unknown')})")
+
+
+def router(x, router_w, k: int, bias=None):
+    """Steps 1-4 (C oracle).  Returns (logits [B,E] f64, ids [B,k] i32, w [B,k] f64)."""
+    lib = _load()
+    x = _u16(x)
+    router_w = _u16(router_w)
+    B, H = x.shape
+    H2, E = router_w.shape
+    assert H == H2
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    logits = np.zeros((B, E), np.float64)
+    ids = np.zeros((B, k), np.int32)
+    w = np.zeros((B, k), np.float64)
+    _check(lib.oracle_router(_ptr(x), _ptr(router_w), _ptr(b), B, H, E, k,
+                             _ptr(logits), _ptr(ids), _ptr(w)), "oracle_router")
+    return logits, ids, w
+
+
+def block(x, ids, w, w13: Sequence, w2: Sequence, sw13=None, sw2=None, n_experts=None):
+    """Steps 5-7 (C oracle) for a given routing.  ``w13``/``w2`` are sequences of
+    length E (entries for experts that are never selected may be None)."""
+    lib = _load()
+    x = _u16(x)
+    B, H = x.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    k = ids.shape[1] if ids.ndim == 2 else 0
+    E = len(w13) if n_experts is None else n_experts
+    keep = []
+    arr13 = (ctypes.c_void_p * E)()
+    arr2 = (ctypes.c_void_p * E)()
+    inter = None
+    for e in range(E):
+        if w13[e] is not None:
+            a13 = _u16(w13[e]); a2 = _u16(w2[e])
+            keep += [a13, a2]
+            arr13[e] = a13.ctypes.data
+            arr2[e] = a2.ctypes.data
+            inter = a13.shape[1] // 2
+    if inter is None:
+        raise ValueError("no expert weights given")
+    n_shared = 0 if sw13 is None else 1
+    Is = 0
+    if n_shared:
+        sw13 = _u16(sw13); sw2 = _u16(sw2)
+        Is = sw13.shape[1] // 2
+    out = np.zeros((B, H), np.float64)
+    _check(lib.oracle_block(_ptr(x), _ptr(ids), _ptr(w), arr13, arr2, _ptr(sw13), _ptr(sw2),
+                            B, H, E, k, inter, Is, n_shared, _ptr(out)), "oracle_block")
+    del keep
+    return out
+
+
+def moe_forward(x, router_w, w13, w2, sw13, sw2, k: int, bias=None):
+    """Steps 1-7 (C oracle).  Returns (out [B,H] f64, ids, w, logits)."""
+    logits, ids, w = router(x, router_w, k, bias)
+    out = block(x, ids, w, w13, w2, sw13, sw2)
+    return out, ids, w, logits
+
+
+def topk_margin(logits: np.ndarray, k: int) -> np.ndarray:
+    """Smallest gap between consecutive sorted logits among each row's top k+1
+    (used by tests to reject inputs whose top-k order is not well separated)."""
+    s = -np.sort(-logits, axis=1)[:, : k + 1]
+    return np.min(s[:, :-1] - s[:, 1:], axis=1)
