@@ -1,0 +1,210 @@
+/*
+ * moe_decode.h -- C ABI of the B200 (sm_100a) MoE decode-block library.
+ *
+ * One call of moe_decode_forward runs the decode pass of one
+ * Mixture-of-Experts block for a batch of 1..64 tokens on one GPU:
+ *
+ *   1. router scores  logit = x . R (+ bias), softmax over all experts,
+ *      top-k selection (logit descending, ties to the smaller id) and
+ *      renormalisation of the k selected probabilities;
+ *   2. bucketing of the token->expert assignments by expert;
+ *   3. per selected expert, the SwiGLU up projection
+ *      a = silu(x . W13[:, :I]) * (x . W13[:, I:]);
+ *   4. the down projection y = a . W2, weighted by the routing weight;
+ *   5. the shared expert (same MLP, weight 1) on the auxiliary stream;
+ *   6. out = x + sum_j w_j y_j + shared, rounded once to bf16.
+ *
+ * The steps follow the pages "Hyper Optimizing Kimi K3 in vLLM: Moving Fast
+ * and Responsibly" (commentary; section "Recovering time between operators":
+ * small-matrix projection kernels at batch 1-2, split work at larger
+ * batches, the shared expert on another stream, weights prefetched before
+ * their consumer starts) and "vLLM Hyper-Optimizes Kimi K3 on NVIDIA GB300"
+ * (section "What's Optimized": batch-dependent kernels, MoE scheduling,
+ * weight prefetch).  The pages name the steps but give no formulas; the
+ * formulas above are the plainest standard reading (softmax router,
+ * renormalised top-k, SwiGLU with the gate in the first half of w13, one
+ * shared expert of weight 1, residual = the block input x).
+ *
+ * Conventions for every entry point:
+ *   - Return value: MOE_OK (0) or a negative MOE_ERR_* code.  Argument errors
+ *     are detected on the host before anything is enqueued.
+ *   - Tensors are row-major bf16 (IEEE binary32 upper halves) unless stated.
+ *   - "device" pointers point to memory of the GPU the handle was created
+ *     on; "host" pointers to CPU memory.  The caller owns every tensor; the
+ *     library owns its handle, its workspace and its events.
+ *   - Weights are read-only and must not change while a forward that uses
+ *     them may be running.
+ *   - A handle must not run two forwards at the same time (it owns one
+ *     workspace); use one handle per concurrent stream pair.
+ */
+#ifndef MOE_DECODE_H_
+#define MOE_DECODE_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------ error codes */
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)       /* NULL pointer, bad batch, misaligned pointer */
+#define MOE_ERR_UNSUPPORTED_SHAPE (-2) /* shapes outside the supported envelope */
+#define MOE_ERR_NO_DEVICE (-3)         /* no CUDA device visible */
+#define MOE_ERR_ARCH (-4)              /* device is not compute capability 10.x (B200) */
+#define MOE_ERR_CUDA (-5)              /* a CUDA runtime call failed; see moe_decode_last_cuda_error */
+#define MOE_ERR_OUT_OF_MEMORY (-6)     /* workspace allocation failed in init */
+#define MOE_ERR_DEVICE_TIMEOUT (-7)    /* a bounded device-side wait gave up (status word) */
+#define MOE_ERR_DEVICE_PLAN (-8)       /* device-side consistency check failed (status word) */
+
+/* ---------------------------------------------------------------- shapes */
+/*
+ * Block shape, fixed for the life of a handle.  Supported envelope:
+ *   hidden      : multiple of 8, 8..16384
+ *   n_experts   : multiple of 8, 8..1024
+ *   top_k       : 1..min(32, n_experts)
+ *   inter       : multiple of 8, 8..16384 (routed expert intermediate size I)
+ *   shared_inter: multiple of 8, 8..16384 when n_shared == 1 (ignored otherwise)
+ *   n_shared    : 0 or 1
+ *   max_batch   : 1..64; sizes the workspace, forward accepts batch <= max_batch
+ * router_bias (optional) is a device float32 [n_experts] added to the router
+ * logits before softmax and selection; NULL means no bias.  It is read by
+ * every forward (the pointer is kept, the data is not copied).
+ * flags is reserved and must be 0.
+ */
+typedef struct moe_decode_shapes {
+  int32_t hidden;
+  int32_t n_experts;
+  int32_t top_k;
+  int32_t inter;
+  int32_t shared_inter;
+  int32_t n_shared;
+  int32_t max_batch;
+  const float* router_bias;
+  uint32_t flags;
+} moe_decode_shapes;
+
+typedef struct moe_decode_ctx* moe_decode_t;
+
+/*
+ * Per-handle counters (host side), filled by moe_decode_get_stats.
+ *   forwards           : successful moe_decode_forward* calls
+ *   kernels_launched   : kernels enqueued by this handle since creation
+ *   last_kernels       : kernels enqueued by the last forward
+ *   last_variant       : token-group width of the routed expert kernels used
+ *                        by the last forward (1, 2, 4 or 8; 0 = batch 0)
+ *   variant_calls[4]   : forwards per token-group width 1, 2, 4, 8
+ */
+typedef struct moe_decode_stats {
+  uint64_t forwards;
+  uint64_t kernels_launched;
+  int32_t last_kernels;
+  int32_t last_variant;
+  uint64_t variant_calls[4];
+} moe_decode_stats;
+
+/*
+ * Create a handle on the current CUDA device: validates the shapes, checks
+ * the device (compute capability 10.x), allocates and zeroes the workspace
+ * (sized for shapes->max_batch) and creates the fork/join events.  This is
+ * the only entry point that allocates device memory.
+ * shapes: host pointer, read during the call only.  out_handle: host pointer
+ * that receives the handle (set to NULL on error).
+ */
+int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle);
+
+/*
+ * Enqueue one forward of the block on stream_main / stream_aux (cudaStream_t
+ * passed as void*; NULL is the legacy default stream).  Asynchronous, does no
+ * host synchronisation and allocates nothing, so it can be captured in a
+ * CUDA graph.  The shared expert is forked onto stream_aux with an event and
+ * joined back; when the call returns every piece of work is ordered before
+ * anything later enqueued on stream_main.  stream_aux may equal stream_main.
+ *
+ *   x          device bf16 [batch, hidden]          block input and residual
+ *   router_w   device bf16 [hidden, n_experts]      router weights (in x out)
+ *   w13        HOST array of n_experts device pointers; w13[e] -> bf16
+ *              [hidden, 2*inter], columns [0,inter) gate, [inter,2*inter) up
+ *   w2         HOST array of n_experts device pointers; w2[e] -> bf16
+ *              [inter, hidden]
+ *   shared_w13 device bf16 [hidden, 2*shared_inter] (NULL iff n_shared == 0)
+ *   shared_w2  device bf16 [shared_inter, hidden]   (NULL iff n_shared == 0)
+ *   out        device bf16 [batch, hidden]          must not alias x
+ *   topk_ids   device int32 [batch, top_k]          selected experts, best first
+ *   topk_w     device float32 [batch, top_k]        renormalised weights
+ *   batch      0..max_batch (0 enqueues nothing and returns MOE_OK)
+ * The host pointer arrays are read during the call only.  Every device
+ * pointer must be 16-byte aligned; w13[e]/w2[e] must be non-NULL for every
+ * expert (any of them may be selected).
+ * Errors: MOE_ERR_INVALID_ARG for NULL/misaligned pointers or a bad batch,
+ * MOE_ERR_CUDA if a launch fails (the handle's workspace is then re-zeroed
+ * by the next forward).
+ */
+int moe_decode_forward(moe_decode_t h, const void* x, const void* router_w,
+                       const void* const* w13, const void* const* w2,
+                       const void* shared_w13, const void* shared_w2, void* out,
+                       int32_t* topk_ids, float* topk_w, int32_t batch,
+                       void* stream_main, void* stream_aux);
+
+/*
+ * Same computation with the per-step tensors in HOST memory: copies x_host
+ * (bf16 [batch, hidden]) to the handle's device staging buffer, runs the
+ * forward, copies out/topk_ids/topk_w back to out_host/ids_host/w_host and
+ * synchronises stream_main before returning.  Weights stay device pointers.
+ * Pinned host buffers give the fastest copies; pageable ones work.
+ */
+int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* router_w,
+                            const void* const* w13, const void* const* w2,
+                            const void* shared_w13, const void* shared_w2,
+                            void* out_host, int32_t* ids_host, float* w_host,
+                            int32_t batch, void* stream_main, void* stream_aux);
+
+/* Free the workspace and events; NULL is accepted.  Synchronises the device
+ * work of the handle first. */
+int moe_decode_destroy(moe_decode_t h);
+
+/*
+ * Synchronise the handle's device, read and clear its device status word.
+ * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded device wait gave up) or
+ * MOE_ERR_DEVICE_PLAN (a device consistency check failed), or MOE_ERR_CUDA.
+ */
+int moe_decode_get_status(moe_decode_t h);
+
+/* Copy the handle's counters to *stats (host pointer). */
+int moe_decode_get_stats(moe_decode_t h, moe_decode_stats* stats);
+
+/* Static string for a MOE_* code; never NULL. */
+const char* moe_decode_error_string(int code);
+
+/* The last CUDA error seen by any entry point of this thread (cudaError_t
+ * value, 0 if none) and its name. */
+int moe_decode_last_cuda_error(void);
+const char* moe_decode_last_cuda_error_string(void);
+
+/*
+ * Per-kernel timing.  events: HOST array of MOE_TIMING_EVENTS cudaEvent_t
+ * (passed as void*) created by the caller with timing enabled, or NULL to
+ * switch timing off.  While set, every forward records, on stream_main,
+ *   [0] before the router, [1] after the router, [2] after the routed up
+ *   projection, [3] after the routed down projection, [4] after the combine,
+ * and on stream_aux
+ *   [5] before the shared up projection, [6] after it, [7] after the shared
+ *   down projection,
+ * so cudaEventElapsedTime gives each kernel's duration.  Recording an event
+ * between two kernels also makes the second wait for the first to finish
+ * (no early launch), so timed forwards can be slightly slower.  The handle
+ * keeps the array's values (not the pointer); the caller keeps the events
+ * alive while timing is on.
+ */
+#define MOE_TIMING_EVENTS 8
+int moe_decode_set_timing_events(moe_decode_t h, void* const* events, int32_t n_events);
+
+/* Workspace bytes that moe_decode_init would allocate for these shapes (0 if
+ * the shapes are invalid).  Pure host computation. */
+uint64_t moe_decode_workspace_bytes(const moe_decode_shapes* shapes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DECODE_H_ */

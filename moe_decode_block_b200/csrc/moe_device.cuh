@@ -1,0 +1,154 @@
+// moe_device.cuh -- device-side building blocks shared by the MoE decode
+// kernels: constants, the routing plan written by the router kernel, and
+// thin wrappers over the sm_90+/sm_100 PTX used for TMA bulk staging
+// (cp.async.bulk + mbarrier), L2 prefetch and bounded waits.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kMaxBatch = 64;
+constexpr int kMaxAssign = kMaxBatch * kMaxTopK;
+
+// Expert GEMV kernels: 16 consumer warps own one 16-byte column vector each
+// (8 bf16 columns), one producer warp issues the TMA bulk copies.
+constexpr int kConsumerWarps = 16;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kGemvThreads = kConsumerThreads + 32;
+constexpr int kMaxPanelCols = 8 * kConsumerThreads;  // local columns per panel
+constexpr int kStepRows = 64;    // rows per partition step (and per activation chunk)
+constexpr int kStageBytes = 32 * 1024;
+constexpr int kMaxStages = 8;
+
+constexpr int kRouterThreads = 256;
+
+// Device status word values (the host maps them to MOE_ERR_*).
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusPlan = 2;
+
+// Bounded-wait limit: try_wait already suspends in hardware for a while per
+// probe, so this bounds a stuck wait to well under a minute.
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+// Routing plan: written by the last router CTA, read by the expert kernels.
+// Units are the active experts in ascending id order; the assignments of
+// unit u are [unit_begin[u], unit_begin[u] + unit_count[u]) sorted by token.
+struct Plan {
+  int n_active;
+  int pad_[3];
+  int unit_expert[kMaxExperts];
+  int unit_begin[kMaxExperts];
+  int unit_count[kMaxExperts];
+  int assign_tok[kMaxAssign];   // token index b
+  int assign_slot[kMaxAssign];  // b * top_k + j (row of the per-assignment buffers)
+  float assign_w[kMaxAssign];   // renormalised routing weight
+};
+
+// Per-expert weight pointers, passed by value as a __grid_constant__
+// parameter (8 KB) so no per-call host->device copy is needed.
+struct ExpertTable {
+  const __nv_bfloat16* p[kMaxExperts];
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+
+// Make mbarrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Wait for the phase of `bar` with the given parity; gives up after
+// kSpinLimit probes, records kStatusTimeout in *status and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  atomicCAS(status, kStatusOk, kStatusTimeout);
+  return false;
+}
+
+// Same, for waits inside a CTA that shares an abort flag: once any thread
+// of the CTA has given up, the others stop waiting within ~1k probes, so a
+// failed copy never turns into a hang.  Callers keep executing the same
+// barrier sequence after a failure (skipping only the work).
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t parity, int* status,
+                                                    volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023u) == 1023u && *abort_flag) return false;
+  }
+  atomicCAS(status, kStatusOk, kStatusTimeout);
+  *abort_flag = 1;
+  return false;
+}
+
+// L2 policy for weight streams: each weight byte is read once per forward,
+// so mark it evict-first and leave L2 to the small activation buffers.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// TMA bulk copy global -> shared (no multicast), completion counted on `bar`.
+// dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// Bulk prefetch of a global range into L2 (no data returned to the SM).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Named barrier over the consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
+}
+
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t v, float& lo, float& hi) {
+  lo = __uint_as_float(v << 16);
+  hi = __uint_as_float(v & 0xffff0000u);
+}
+
+__device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
+
+}  // namespace moe

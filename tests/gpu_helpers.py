@@ -1,0 +1,91 @@
+"""Shared helpers for the GPU parity tests: seeded inputs with a top-k logit
+margin (checked with the oracle's router on the host) and comparison of the
+CUDA path against the fp64 oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from moe_decode_block_b200 import MoEDecode, synth
+
+OUT_RTOL = 2e-2      # max|out - oracle| <= 2e-2 * rms(oracle out)
+W_ATOL = 1e-5        # |topk_w - oracle| (fp32 softmax vs fp64)
+MIN_MARGIN = 1e-3    # top-(k+1) logit gaps of every generated row
+
+
+def bias_np(wts):
+    return None if wts.router_bias is None else wts.router_bias.detach().float().cpu().numpy()
+
+
+def margin_x(batch, hidden, wts, k, seed=0, device="cuda", min_gap=MIN_MARGIN):
+    """x [batch, hidden] whose rows all have top-(k+1) logit gaps >= min_gap
+    (fp64 logits of the bf16 values); failing rows are redrawn."""
+    attempts = np.zeros(batch, dtype=np.int64)
+    rb = synth.bf16_bits(wts.router_w)
+    bias = bias_np(wts)
+    for _ in range(64):
+        x = synth.make_x(batch, hidden, seed=seed, attempts=attempts)
+        if batch == 0:
+            return x.to(device)
+        logits, _, _ = oracle.router(synth.bf16_bits(x), rb, k, bias)
+        bad = oracle.topk_margin(logits, k) < min_gap
+        if not bad.any():
+            return x.to(device)
+        attempts[bad] += 1
+    raise RuntimeError("could not draw inputs with the required top-k margin")
+
+
+class Run:
+    """Device buffers and one handle for a block shape."""
+
+    def __init__(self, shape: synth.BlockShape, wts, max_batch=64):
+        self.s = shape
+        self.wts = wts
+        self.blk = MoEDecode(shape.hidden, shape.n_experts, shape.top_k, shape.inter, shape.shared_inter,
+                             n_shared=shape.n_shared, max_batch=max_batch, router_bias=wts.router_bias)
+
+    def forward(self, x, stream_aux=None, w13=None, w2=None):
+        B = x.shape[0]
+        k = self.s.top_k
+        out = torch.full_like(x, float("nan"))
+        ids = torch.full((B, k), -1, dtype=torch.int32, device=x.device)
+        w = torch.full((B, k), float("nan"), dtype=torch.float32, device=x.device)
+        self.blk.forward(x, self.wts.router_w, self.wts.w13 if w13 is None else w13,
+                         self.wts.w2 if w2 is None else w2, self.wts.shared_w13, self.wts.shared_w2,
+                         out, ids, w, stream_aux=stream_aux)
+        torch.cuda.synchronize()
+        return out, ids, w
+
+
+def oracle_check(wts, k, x, out, ids, w, rows=None, w13=None, w2=None):
+    """ids exact and weights within W_ATOL for every row; outputs of `rows`
+    (all rows by default) within OUT_RTOL * rms against the fp64 oracle."""
+    xb = synth.bf16_bits(x)
+    o_logits, o_ids, o_w = oracle.router(xb, synth.bf16_bits(wts.router_w), k, bias_np(wts))
+    g_ids = ids.cpu().numpy()
+    np.testing.assert_array_equal(g_ids, o_ids)
+    g_w = w.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(g_w - o_w), initial=0.0) <= W_ATOL
+    assert np.max(np.abs(g_w.sum(axis=1) - 1.0), initial=0.0) <= 1e-6
+    if rows is None:
+        rows = np.arange(x.shape[0])
+    rows = np.asarray(rows)
+    W13 = wts.w13 if w13 is None else w13
+    W2 = wts.w2 if w2 is None else w2
+    E = wts.router_w.shape[1]
+    need = sorted(set(o_ids[rows].ravel().tolist()))
+    h13 = [None] * E
+    h2 = [None] * E
+    for e in need:
+        h13[e] = synth.bf16_bits(W13[e])
+        h2[e] = synth.bf16_bits(W2[e])
+    sw13 = None if wts.shared_w13 is None else synth.bf16_bits(wts.shared_w13)
+    sw2 = None if wts.shared_w2 is None else synth.bf16_bits(wts.shared_w2)
+    o_out = oracle.block(xb[rows], o_ids[rows], o_w[rows], h13, h2, sw13, sw2, n_experts=E)
+    g_out = out.float().cpu().numpy()[rows]
+    err = np.abs(g_out - o_out)
+    rms = float(np.sqrt(np.mean(o_out ** 2)))
+    assert np.all(np.isfinite(g_out))
+    assert err.max() <= OUT_RTOL * rms, f"max|err| {err.max():.4g} > {OUT_RTOL} * rms {rms:.4g}"
+    return float(err.max()), rms
