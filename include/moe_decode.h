@@ -132,7 +132,8 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle);
  *   out        device bf16 [batch, hidden]          must not alias x
  *   topk_ids   device int32 [batch, top_k]          selected experts, best first
  *   topk_w     device float32 [batch, top_k]        renormalised weights
- *   batch      0..max_batch (0 enqueues nothing and returns MOE_OK)
+ *   batch      0..max_batch (0 enqueues nothing, reads no pointer other
+ *              than the handle and returns MOE_OK)
  * The host pointer arrays are read during the call only.  Every device
  * pointer must be 16-byte aligned; w13[e]/w2[e] must be non-NULL for every
  * expert (any of them may be selected).

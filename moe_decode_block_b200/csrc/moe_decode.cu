@@ -378,6 +378,7 @@ int check_forward_args(moe_decode_ctx* h, const void* x, const void* router_w, c
   if (!h) return MOE_ERR_INVALID_ARG;
   const moe_decode_shapes& s = h->s;
   if (batch < 0 || batch > s.max_batch) return MOE_ERR_INVALID_ARG;
+  if (batch == 0) return MOE_OK;  // nothing is read or written
   if (!x || !router_w || !w13 || !w2 || !out || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
   if (device_io) {
     if (!aligned16(x) || !aligned16(out) || !aligned4(topk_ids) || !aligned4(topk_w)) return MOE_ERR_INVALID_ARG;
