@@ -200,6 +200,45 @@ const char* moe_decode_last_cuda_error_string(void);
 #define MOE_TIMING_EVENTS 8
 int moe_decode_set_timing_events(moe_decode_t h, void* const* events, int32_t n_events);
 
+/*
+ * Router step only (scores, softmax, top-k, renormalised weights) without a
+ * handle and without allocating anything.  The pages have no counterpart for
+ * this entry point; it exists for callers that may not call cudaMalloc at all
+ * -- for example code that runs while a CUDA graph is being captured, or a
+ * host framework that owns every device allocation through its own pool and
+ * forbids plug-ins from allocating behind its back -- and so cannot create a
+ * handle with moe_decode_init.
+ *
+ *   x          device bf16 [batch, hidden]
+ *   router_w   device bf16 [hidden, n_experts]
+ *   router_bias device float32 [n_experts] or NULL
+ *   topk_ids   device int32 [batch, top_k]  (selected experts, best first)
+ *   topk_w     device float32 [batch, top_k] (renormalised weights)
+ *   stream     cudaStream_t as void* (NULL = legacy default stream)
+ * Results equal those of moe_decode_forward for the same inputs.
+ *
+ * Scratch: a fixed static device array of about 300 KB inside this library
+ * (held by every GPU that loads it until the process exits), which bounds the
+ * sizes: batch <= MOE_NOALLOC_MAX_BATCH, n_experts <= MOE_NOALLOC_MAX_EXPERTS
+ * (plus the limits of moe_decode_shapes); larger sizes return
+ * MOE_ERR_UNSUPPORTED_SHAPE.  batch 0 returns MOE_OK without reading any
+ * pointer.  The first call on a device does a one-time set-up (looks up the
+ * array's device address, zeroes it with a synchronous memset), so make that
+ * first call before any stream capture.  Every call clears the part of the
+ * array that must start at zero with cudaMemsetAsync on `stream` and then
+ * launches one kernel; it calls no cudaMalloc, cudaFree or allocating library
+ * routine.  All calls on a device share the one array: calls that may
+ * overlap on the GPU (different streams without ordering between them) race
+ * and must not be issued; calls on one stream are ordered and safe.
+ * Errors: MOE_ERR_UNSUPPORTED_SHAPE, MOE_ERR_INVALID_ARG (NULL or misaligned
+ * pointers), MOE_ERR_ARCH, MOE_ERR_CUDA.
+ */
+#define MOE_NOALLOC_MAX_BATCH 64
+#define MOE_NOALLOC_MAX_EXPERTS 1024
+int moe_router_topk_noalloc(const void* x, const void* router_w, const float* router_bias,
+                            int32_t* topk_ids, float* topk_w, int32_t batch, int32_t hidden,
+                            int32_t n_experts, int32_t top_k, void* stream);
+
 /* Workspace bytes that moe_decode_init would allocate for these shapes (0 if
  * the shapes are invalid).  Pure host computation. */
 uint64_t moe_decode_workspace_bytes(const moe_decode_shapes* shapes);

@@ -32,7 +32,7 @@ EXPORTED = (
     "moe_decode_init", "moe_decode_forward", "moe_decode_forward_host", "moe_decode_destroy",
     "moe_decode_get_status", "moe_decode_get_stats", "moe_decode_error_string",
     "moe_decode_last_cuda_error", "moe_decode_last_cuda_error_string", "moe_decode_workspace_bytes",
-    "moe_decode_set_timing_events",
+    "moe_decode_set_timing_events", "moe_router_topk_noalloc",
 )
 MOE_TIMING_EVENTS = 8
 
@@ -98,6 +98,9 @@ def load_library() -> ctypes.CDLL:
     lib.moe_decode_last_cuda_error_string.restype = ctypes.c_char_p
     lib.moe_decode_set_timing_events.argtypes = [P, P, ctypes.c_int32]
     lib.moe_decode_set_timing_events.restype = I
+    lib.moe_router_topk_noalloc.argtypes = [P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                            ctypes.c_int32, P]
+    lib.moe_router_topk_noalloc.restype = I
     lib.moe_decode_workspace_bytes.argtypes = [ctypes.POINTER(Shapes)]
     lib.moe_decode_workspace_bytes.restype = ctypes.c_uint64
     _lib = lib
@@ -123,6 +126,20 @@ def _stream_handle(s) -> Optional[int]:
     if isinstance(s, int):
         return s
     return s.cuda_stream
+
+
+def router_topk_noalloc(x, router_w, topk_ids, topk_w, top_k: int, router_bias=None, stream=None):
+    """Router scores, softmax, top-k and renormalised weights without a handle
+    and without any device allocation (moe_router_topk_noalloc).  Make the
+    first call on a device outside stream capture; calls that may overlap on
+    the GPU share one scratch array and race."""
+    import torch
+    lib = load_library()
+    sm = _stream_handle(stream if stream is not None else torch.cuda.current_stream())
+    rc = lib.moe_router_topk_noalloc(_ptr(x), _ptr(router_w), _ptr(router_bias), _ptr(topk_ids), _ptr(topk_w),
+                                     int(x.shape[0]), int(router_w.shape[0]), int(router_w.shape[1]), int(top_k),
+                                     sm)
+    _check(rc, "moe_router_topk_noalloc")
 
 
 class MoEDecode:

@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "moe_decode.h"
@@ -414,7 +415,125 @@ struct DeviceGuard {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Router + top-k without a handle and without any allocation.
+//
+// Its scratch (status word, ticket, fp32 logit accumulators for up to
+// MOE_NOALLOC_MAX_BATCH x MOE_NOALLOC_MAX_EXPERTS, and the bucketing plan
+// the kernel also writes) lives in the file-scope device array below, which
+// every GPU that loads this library keeps until the process exits (~300 KB).
+// Host code must not hand the array's name to a kernel -- on the host it is
+// only a stand-in -- so the device address is looked up once per device with
+// cudaGetSymbolAddress and cached.
+namespace {
+
+constexpr size_t kNoAllocLogitsOff = 256;  // bytes [0,4): status, [4,8): ticket
+constexpr size_t kNoAllocPlanOff =
+    kNoAllocLogitsOff + (size_t)MOE_NOALLOC_MAX_BATCH * MOE_NOALLOC_MAX_EXPERTS * sizeof(float);
+constexpr size_t kNoAllocBytes = (kNoAllocPlanOff + sizeof(Plan) + 255) / 256 * 256;
+constexpr int kNoAllocMaxDevices = 64;
+
+struct NoAllocDevice {
+  bool ready = false;
+  uint8_t* scratch = nullptr;
+  int num_sms = 0;
+};
+
+std::mutex g_noalloc_mu;
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_router_scratch[kNoAllocBytes];
+
+namespace {
+
+// First call on a device: resolve the scratch address, zero it once, read the
+// SM count.  Runs with `dev` current.
+int noalloc_setup(int dev, NoAllocDevice** out) {
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoAllocDevice& d = g_noalloc_dev[dev];
+  if (!d.ready) {
+    int major = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return fail_cuda(e);
+    if (major != 10) return MOE_ERR_ARCH;
+    void* p = nullptr;
+    if ((e = cudaGetSymbolAddress(&p, g_router_scratch)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaMemset(p, 0, kNoAllocBytes)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return fail_cuda(e);
+    d.scratch = static_cast<uint8_t*>(p);
+    d.ready = true;
+  }
+  *out = &d;
+  return MOE_OK;
+}
+
+}  // namespace
+
 extern "C" {
+
+int moe_router_topk_noalloc(const void* x, const void* router_w, const float* router_bias, int32_t* topk_ids,
+                            float* topk_w, int32_t batch, int32_t hidden, int32_t n_experts, int32_t top_k,
+                            void* stream) {
+  if (batch < 0 || batch > MOE_NOALLOC_MAX_BATCH) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (hidden < 8 || hidden > 16384 || hidden % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (n_experts < 8 || n_experts > MOE_NOALLOC_MAX_EXPERTS || n_experts % 8) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (top_k < 1 || top_k > moe::kMaxTopK || top_k > n_experts) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (batch == 0) return MOE_OK;
+  if (!x || !router_w || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(router_w) || !aligned4(topk_ids) || !aligned4(topk_w)) return MOE_ERR_INVALID_ARG;
+  if (router_bias && !aligned4(router_bias)) return MOE_ERR_INVALID_ARG;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  NoAllocDevice* d = nullptr;
+  int rc = noalloc_setup(dev, &d);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // The scratch keeps the previous call's contents: the status word, the
+  // ticket and this call's logit accumulators must start at zero.
+  const size_t clear = kNoAllocLogitsOff + (size_t)batch * n_experts * sizeof(float);
+  if ((e = cudaMemsetAsync(d->scratch, 0, clear, st)) != cudaSuccess) return fail_cuda(e);
+
+  RouterArgs ra{};
+  ra.x = static_cast<const __nv_bfloat16*>(x);
+  ra.router_w = static_cast<const __nv_bfloat16*>(router_w);
+  ra.bias = router_bias;
+  ra.B = batch;
+  ra.H = hidden;
+  ra.E = n_experts;
+  ra.k = top_k;
+  int g = d->num_sms < hidden / 8 ? d->num_sms : hidden / 8;
+  if (batch > 8) {
+    const int cap = d->num_sms * 8 / batch;
+    g = g < cap ? g : cap;
+  }
+  ra.G = g < 1 ? 1 : g;
+  const int rows = ceil_div(hidden, ra.G);
+  const int cap_rows = 40960 / (2 * n_experts);
+  ra.chunk_rows = rows < cap_rows ? rows : cap_rows;
+  if (ra.chunk_rows < 1) ra.chunk_rows = 1;
+  ra.status = reinterpret_cast<int*>(d->scratch);
+  ra.ticket = reinterpret_cast<unsigned*>(d->scratch + 4);
+  ra.logits = reinterpret_cast<float*>(d->scratch + kNoAllocLogitsOff);
+  ra.plan = reinterpret_cast<Plan*>(d->scratch + kNoAllocPlanOff);
+  ra.topk_ids = topk_ids;
+  ra.topk_w = topk_w;
+  const size_t smem = moe::router_smem_bytes(batch, n_experts, ra.chunk_rows);
+  cudaFuncAttributes fa{};
+  if ((e = cudaFuncGetAttributes(&fa, moe::router_topk_kernel)) != cudaSuccess) return fail_cuda(e);
+  if ((size_t)fa.maxDynamicSharedSizeBytes < smem) {
+    e = cudaFuncSetAttribute(moe::router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return fail_cuda(e);
+  }
+  e = launch(moe::router_topk_kernel, ra.G, moe::kRouterThreads, smem, st, false, ra);
+  if (e != cudaSuccess) return fail_cuda(e);
+  return MOE_OK;
+}
 
 uint64_t moe_decode_workspace_bytes(const moe_decode_shapes* shapes) {
   if (!shapes_valid(shapes)) return 0;

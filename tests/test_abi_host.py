@@ -23,7 +23,7 @@ def lib():
 def header_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(moe_decode_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moe_\w+)\s*\(", text)))
 
 
 def test_header_declares_the_binding_names():
