@@ -88,19 +88,18 @@ typedef struct moe_decode_ctx* moe_decode_t;
 
 /*
  * Per-handle counters (host side), filled by moe_decode_get_stats.
- *   forwards           : successful moe_decode_forward* calls
- *   kernels_launched   : kernels enqueued by this handle since creation
- *   last_kernels       : kernels enqueued by the last forward
- *   last_variant       : token-group width of the routed expert kernels used
- *                        by the last forward (1, 2, 4 or 8; 0 = batch 0)
- *   variant_calls[4]   : forwards per token-group width 1, 2, 4, 8
+ *   forwards          : successful forwards enqueued by this handle
+ *   kernels_launched  : kernels enqueued by this handle since creation
+ *   last_kernels      : kernels enqueued by the last forward (4, or 3 without
+ *                       a shared expert)
+ *   last_token_tiles  : token tiles of 8 the expert kernels were prepared for
+ *                       in the last forward (ceil(batch / 8))
  */
 typedef struct moe_decode_stats {
   uint64_t forwards;
   uint64_t kernels_launched;
   int32_t last_kernels;
-  int32_t last_variant;
-  uint64_t variant_calls[4];
+  int32_t last_token_tiles;
 } moe_decode_stats;
 
 /*
@@ -186,18 +185,17 @@ const char* moe_decode_last_cuda_error_string(void);
  * Per-kernel timing.  events: HOST array of MOE_TIMING_EVENTS cudaEvent_t
  * (passed as void*) created by the caller with timing enabled, or NULL to
  * switch timing off.  While set, every forward records, on stream_main,
- *   [0] before the router, [1] after the router, [2] after the routed up
- *   projection, [3] after the routed down projection, [4] after the combine,
+ *   [0] before the router, [1] after the router, [2] after the routed
+ *   experts (up + SwiGLU + down), [3] after the combine,
  * and on stream_aux
- *   [5] before the shared up projection, [6] after it, [7] after the shared
- *   down projection,
+ *   [4] before the shared expert, [5] after it,
  * so cudaEventElapsedTime gives each kernel's duration.  Recording an event
  * between two kernels also makes the second wait for the first to finish
  * (no early launch), so timed forwards can be slightly slower.  The handle
  * keeps the array's values (not the pointer); the caller keeps the events
  * alive while timing is on.
  */
-#define MOE_TIMING_EVENTS 8
+#define MOE_TIMING_EVENTS 6
 int moe_decode_set_timing_events(moe_decode_t h, void* const* events, int32_t n_events);
 
 /*

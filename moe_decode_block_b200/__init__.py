@@ -34,7 +34,7 @@ EXPORTED = (
     "moe_decode_last_cuda_error", "moe_decode_last_cuda_error_string", "moe_decode_workspace_bytes",
     "moe_decode_set_timing_events", "moe_router_topk_noalloc",
 )
-MOE_TIMING_EVENTS = 8
+MOE_TIMING_EVENTS = 6
 
 
 class Shapes(ctypes.Structure):
@@ -48,8 +48,7 @@ class Shapes(ctypes.Structure):
 class Stats(ctypes.Structure):
     _fields_ = [
         ("forwards", ctypes.c_uint64), ("kernels_launched", ctypes.c_uint64),
-        ("last_kernels", ctypes.c_int32), ("last_variant", ctypes.c_int32),
-        ("variant_calls", ctypes.c_uint64 * 4),
+        ("last_kernels", ctypes.c_int32), ("last_token_tiles", ctypes.c_int32),
     ]
 
 
@@ -213,7 +212,7 @@ class MoEDecode:
         _check(rc, "moe_decode_forward_host")
 
     def set_timing_events(self, events):
-        """Record per-kernel CUDA events in every forward (list of 8
+        """Record per-kernel CUDA events in every forward (list of 6
         torch.cuda.Event(enable_timing=True)), or stop with None."""
         if events is None:
             _check(self._lib.moe_decode_set_timing_events(self._h, None, 0), "moe_decode_set_timing_events")
@@ -236,7 +235,7 @@ class MoEDecode:
         s = Stats()
         _check(self._lib.moe_decode_get_stats(self._h, ctypes.byref(s)), "moe_decode_get_stats")
         return {"forwards": s.forwards, "kernels_launched": s.kernels_launched, "last_kernels": s.last_kernels,
-                "last_variant": s.last_variant, "variant_calls": list(s.variant_calls)}
+                "last_token_tiles": s.last_token_tiles}
 
     def close(self):
         if getattr(self, "_h", None):

@@ -1,66 +1,48 @@
 // moe_decode.cu -- host side of the C ABI declared in include/moe_decode.h.
 //
-// One forward enqueues six kernels:
-//   stream_aux : shared-expert UP, shared-expert DOWN          (weight 1)
-//   stream_main: router+top-k+plan, routed UP, routed DOWN, [join] combine
+// One forward enqueues four kernels:
+//   stream_main: router+top-k+plan, routed experts (UP + SwiGLU + DOWN), [join] combine
+//   stream_aux : shared expert (UP + SwiGLU + DOWN, weight 1), forked after the router
 // The shared expert is forked from stream_main with an event and joined back
 // before the combine (pages: "Hyper Optimizing Kimi K3 in vLLM", section
 // "Recovering time between operators": the shared expert runs on another
 // stream, overlapping routing and the selected experts).  Consecutive kernels
 // on one stream use programmatic dependent launch so the next kernel's CTAs
 // start (and prefetch static weights) while the previous one drains.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <vector>
 
 #include "moe_decode.h"
-#include "expert_gemv.cuh"
+#include "combine.cuh"
+#include "expert_mma.cuh"
 #include "moe_device.cuh"
 #include "router_topk.cuh"
 
 namespace {
 
 using moe::ExpertTable;
-using moe::GemvArgs;
+using moe::MmaArgs;
 using moe::Plan;
 using moe::RouterArgs;
 
 thread_local int g_last_cuda_error = 0;
 
-struct Geom {
-  int K, N, I, panel_w, n_cp, stage_rows;
-};
-
 struct WorkspaceLayout {
-  size_t status, ticket, logits, plan, h, a, counters, h_s, a_s, counters_s, acc, x_stage, out_stage,
-      ids_stage, w_stage, total;
+  size_t status, ticket, logits, plan, h, a, panel_cnt, panel_ready, queue, h_s, a_s, panel_cnt_s, panel_ready_s,
+      queue_s, acc, x_stage, out_stage, ids_stage, w_stage, maps, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
-
-// Column panels and stage rows of one projection.  UP panels pair gate
-// column c with up column I + c; each panel has at most kMaxPanelCols local
-// columns.  stage_rows is the largest power of two (<= 64) whose rows fit
-// one 32 KB stage.
-Geom make_geom(bool up, int K, int cols) {
-  Geom g{};
-  g.K = K;
-  const int maxw = up ? moe::kMaxPanelCols / 2 : moe::kMaxPanelCols;
-  g.N = up ? 2 * cols : cols;
-  g.I = up ? cols : 0;
-  g.n_cp = ceil_div(cols, maxw);
-  g.panel_w = ceil_div(ceil_div(cols, g.n_cp), 8) * 8;
-  const int lw = up ? 2 * g.panel_w : g.panel_w;
-  int r = moe::kStepRows;
-  while (r > 1 && (size_t)r * lw * 2 > (size_t)moe::kStageBytes) r >>= 1;
-  g.stage_rows = r;
-  return g;
-}
 
 bool shapes_valid(const moe_decode_shapes* s) {
   if (!s) return false;
@@ -76,14 +58,20 @@ bool shapes_valid(const moe_decode_shapes* s) {
   return true;
 }
 
+// Units of a routed pass: one per active expert, plus the extra units of
+// experts routed more than kMaxUnitTokens tokens.
+size_t max_units(const moe_decode_shapes* s) {
+  return (size_t)s->n_experts + ((size_t)s->max_batch * s->top_k) / moe::kMaxUnitTokens;
+}
+
 WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   WorkspaceLayout L{};
   const size_t A = 256;
   const size_t B = (size_t)s->max_batch, E = (size_t)s->n_experts, k = (size_t)s->top_k;
   const size_t H = (size_t)s->hidden, I = (size_t)s->inter;
   const size_t Is = s->n_shared ? (size_t)s->shared_inter : 0;
-  const Geom up = make_geom(true, s->hidden, s->inter);
-  const int ncp_s = s->n_shared ? make_geom(true, s->hidden, s->shared_inter).n_cp : 0;
+  const int ncp = moe::max_up_panels(s->inter);
+  const int ncp_s = s->n_shared ? moe::max_up_panels(s->shared_inter) : 0;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -95,16 +83,22 @@ WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   L.logits = take(B * E * 4);
   L.plan = take(sizeof(Plan));
   L.h = take(B * k * 2 * I * 4);
-  L.a = take(B * k * I * 4);
-  L.counters = take(E * (size_t)up.n_cp * 4);
+  L.a = take(B * k * I * 2);
+  const size_t U = max_units(s);
+  L.panel_cnt = take(U * (size_t)ncp * 4);
+  L.panel_ready = take(U * (size_t)ncp * 4);
+  L.queue = take(4 * 4);
   L.h_s = take(B * 2 * Is * 4);
-  L.a_s = take(B * Is * 4);
-  L.counters_s = take((size_t)ncp_s * 4 + 4);
+  L.a_s = take(B * Is * 2);
+  L.panel_cnt_s = take((size_t)ncp_s * 4 + 4);
+  L.panel_ready_s = take((size_t)ncp_s * 4 + 4);
+  L.queue_s = take(4 * 4);
   L.acc = take(B * H * 4);
   L.x_stage = take(B * H * 2);
   L.out_stage = take(B * H * 2);
   L.ids_stage = take(B * k * 4);
   L.w_stage = take(B * k * 4);
+  L.maps = take((2 * E + 2) * (size_t)moe::kTensorMapBytes);  // tensor maps: w13[E], w2[E], shared w13, w2
   L.total = off;
   return L;
 }
@@ -137,19 +131,59 @@ cudaError_t launch(void (*kern)(KArgs...), int grid, int block, size_t smem, cud
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-using GemvKernel = void (*)(GemvArgs, ExpertTable);
+using MlpKernel = void (*)(MmaArgs, ExpertTable, ExpertTable);
 
-template <bool DENSE, bool UP>
-GemvKernel pick_gemv(int tg) {
-  switch (tg) {
-    case 1: return moe::expert_gemv_kernel<1, DENSE, UP>;
-    case 2: return moe::expert_gemv_kernel<2, DENSE, UP>;
-    case 4: return moe::expert_gemv_kernel<4, DENSE, UP>;
-    default: return moe::expert_gemv_kernel<8, DENSE, UP>;
+// The expert kernel compiled for the largest token class `kc` (0..3) a
+// launch can see, on the tensor-map or the row-copy path.
+template <bool DENSE, bool TMAP>
+MlpKernel pick_mlp_t(int kc) {
+  switch (kc) {
+    case 0: return moe::expert_mlp_kernel<DENSE, 0, TMAP>;
+    case 1: return moe::expert_mlp_kernel<DENSE, 1, TMAP>;
+    case 2: return moe::expert_mlp_kernel<DENSE, 2, TMAP>;
+    default: return moe::expert_mlp_kernel<DENSE, 3, TMAP>;
   }
 }
+template <bool DENSE>
+MlpKernel pick_mlp(int kc, bool tmap) {
+  return tmap ? pick_mlp_t<DENSE, true>(kc) : pick_mlp_t<DENSE, false>(kc);
+}
 
-inline int token_group_for(int n) { return n <= 1 ? 1 : (n <= 2 ? 2 : (n <= 4 ? 4 : 8)); }
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library is needed).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// Tensor map of a row-major bf16 [rows, cols] matrix seen as the 3-D tensor
+// {64 columns, rows, cols / 64 chunks} (strides: one row, 128 bytes), with
+// {64, 16, 4} boxes and 128-byte swizzling (see expert_mma.cuh).
+bool encode_matrix_map(uint8_t* out, const void* base, int rows, int cols) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc || cols % moe::kChunkCols) return false;
+  CUtensorMap m;
+  cuuint64_t dims[3] = {(cuuint64_t)moe::kChunkCols, (cuuint64_t)rows, (cuuint64_t)(cols / moe::kChunkCols)};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)moe::kChunkCols * 2};
+  cuuint32_t box[3] = {(cuuint32_t)moe::kChunkCols, (cuuint32_t)moe::kBoxRows, (cuuint32_t)moe::kBoxChunks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  static_assert(sizeof(CUtensorMap) == moe::kTensorMapBytes, "tensor map size");
+  std::memcpy(out, &m, sizeof m);
+  return true;
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -160,10 +194,10 @@ struct moe_decode_ctx {
   moe_decode_shapes s{};
   int device = 0;
   int num_sms = 0;
-  int n_stages = 6;
+  int n_stages = 3;
   int grid_routed = 0, grid_shared = 0, grid_router_max = 0;
+  bool grid_routed_auto = true;
   int router_chunk_rows = 0;
-  Geom up{}, down{}, sh_up{}, sh_down{};
   WorkspaceLayout L{};
   uint8_t* ws = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
@@ -173,6 +207,13 @@ struct moe_decode_ctx {
   ExpertTable* tab2 = nullptr;
   bool timing = false;
   cudaEvent_t tev[MOE_TIMING_EVENTS] = {};
+  ExpertTable* tab_none = nullptr;  // zero table passed to the shared-expert launch
+  // tensor-map path: maps encoded for the pointer tables of the last forward
+  bool use_tmap = false;
+  uint8_t* maps_host = nullptr;  // pinned staging, (2E + 2) maps
+  std::vector<const void*> map_ptrs;  // w13[E], w2[E], shared w13, shared w2 the maps describe
+  bool maps_uploaded = false;
+  cudaEvent_t ev_maps = nullptr;
 
   template <typename T>
   T* at(size_t off) const {
@@ -192,20 +233,76 @@ int router_grid(const moe_decode_ctx* h, int batch) {
   return g;
 }
 
+// CTAs for the shared expert when it runs beside the routed experts: its
+// share of the forward's weight bytes (routed share estimated for uniform
+// routing, E * (1 - (1 - k/E)^B) distinct experts), scaled up when the batch
+// puts the shared expert in a narrow-panel class whose smaller row copies
+// stream more slowly per SM.  The routed kernel gets the remaining SMs, so the
+// two grids never wait for each other's SMs.
+int shared_grid(const moe_decode_ctx* h, int batch) {
+  if (h->grid_shared > 0) return h->grid_shared;
+  const moe_decode_shapes& s = h->s;
+  const double E = s.n_experts, k = s.top_k;
+  const double distinct = E * (1.0 - std::pow(1.0 - k / E, (double)batch));
+  const double routed = distinct * 3.0 * s.hidden * s.inter;
+  const int cls = moe::class_for_tokens(batch);
+  const double slow = cls <= 1 ? 1.3 : (cls == 2 ? 3.0 : 6.0);
+  const double shared = 3.0 * s.hidden * s.shared_inter * slow;
+  int g = (int)std::ceil(h->num_sms * shared / (shared + routed));
+  const int cap = h->num_sms / 2;
+  g = g < 1 ? 1 : (g > cap ? cap : g);
+  return g;
+}
+
 int set_kernel_attrs(const moe_decode_ctx* h) {
-  const int gemv_smem = (int)moe::gemv_smem_bytes(h->n_stages, 8);
-  GemvKernel ks[] = {
-      pick_gemv<false, true>(1), pick_gemv<false, true>(2), pick_gemv<false, true>(4), pick_gemv<false, true>(8),
-      pick_gemv<false, false>(1), pick_gemv<false, false>(2), pick_gemv<false, false>(4), pick_gemv<false, false>(8),
-      pick_gemv<true, true>(1), pick_gemv<true, true>(2), pick_gemv<true, true>(4), pick_gemv<true, true>(8),
-      pick_gemv<true, false>(1), pick_gemv<true, false>(2), pick_gemv<true, false>(4), pick_gemv<true, false>(8)};
-  for (GemvKernel k : ks) {
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, gemv_smem);
-    if (e != cudaSuccess) return fail_cuda(e);
+  const int smem = (int)moe::mma_smem_bytes(h->n_stages);
+  cudaError_t e;
+  for (int kc = 0; kc < moe::kNumClasses; ++kc) {
+    for (int tm = 0; tm < 2; ++tm) {
+      e = cudaFuncSetAttribute(pick_mlp<false>(kc, tm), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return fail_cuda(e);
+      e = cudaFuncSetAttribute(pick_mlp<true>(kc, tm), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return fail_cuda(e);
+    }
   }
   const int rsmem = (int)moe::router_smem_bytes(h->s.max_batch, h->s.n_experts, h->router_chunk_rows);
-  cudaError_t e = cudaFuncSetAttribute(moe::router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
+  e = cudaFuncSetAttribute(moe::router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
   if (e != cudaSuccess) return fail_cuda(e);
+  return MOE_OK;
+}
+
+// Tensor-map path: (re)encode the maps whose matrices moved since the last
+// forward and copy the table to the workspace, in stream order.  Weight
+// pointers normally stay fixed, so this usually does nothing.
+int refresh_maps(moe_decode_ctx* h, const void* const* w13, const void* const* w2, const void* sw13,
+                 const void* sw2, cudaStream_t sm) {
+  const moe_decode_shapes& s = h->s;
+  const int E = s.n_experts;
+  bool changed = !h->maps_uploaded;
+  for (int e = 0; e < E && !changed; ++e) changed = (h->map_ptrs[e] != w13[e] || h->map_ptrs[E + e] != w2[e]);
+  if (s.n_shared && !changed) changed = (h->map_ptrs[2 * E] != sw13 || h->map_ptrs[2 * E + 1] != sw2);
+  if (!changed) return MOE_OK;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(sm, &cap);
+  // the staging buffer may still feed the previous upload
+  if (h->maps_uploaded && cap == cudaStreamCaptureStatusNone) cudaEventSynchronize(h->ev_maps);
+  const size_t mb = moe::kTensorMapBytes;
+  for (int e = 0; e < E; ++e) {
+    if (!encode_matrix_map(h->maps_host + e * mb, w13[e], s.hidden, 2 * s.inter)) return MOE_ERR_INVALID_ARG;
+    if (!encode_matrix_map(h->maps_host + (E + e) * mb, w2[e], s.inter, s.hidden)) return MOE_ERR_INVALID_ARG;
+    h->map_ptrs[e] = w13[e];
+    h->map_ptrs[E + e] = w2[e];
+  }
+  if (s.n_shared) {
+    if (!encode_matrix_map(h->maps_host + 2 * E * mb, sw13, s.hidden, 2 * s.shared_inter)) return MOE_ERR_INVALID_ARG;
+    if (!encode_matrix_map(h->maps_host + (2 * E + 1) * mb, sw2, s.shared_inter, s.hidden)) return MOE_ERR_INVALID_ARG;
+    h->map_ptrs[2 * E] = sw13;
+    h->map_ptrs[2 * E + 1] = sw2;
+  }
+  cudaError_t e = cudaMemcpyAsync(h->ws + h->L.maps, h->maps_host, (2 * E + 2) * mb, cudaMemcpyHostToDevice, sm);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (cap == cudaStreamCaptureStatusNone && (e = cudaEventRecord(h->ev_maps, sm)) != cudaSuccess) return fail_cuda(e);
+  h->maps_uploaded = true;
   return MOE_OK;
 }
 
@@ -225,10 +322,16 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     h->tab13->p[i] = static_cast<const __nv_bfloat16*>(w13[i]);
     h->tab2->p[i] = static_cast<const __nv_bfloat16*>(w2[i]);
   }
+  if (h->use_tmap) {
+    const int rc = refresh_maps(h, w13, w2, shared_w13, shared_w2, sm);
+    if (rc != MOE_OK) return rc;
+  }
+  const uint8_t* maps = h->ws + h->L.maps;
+  const size_t mb = moe::kTensorMapBytes;
   int* status = h->at<int>(h->L.status);
   float* acc = h->at<float>(h->L.acc);
   const bool fork = s.n_shared && sa != sm;
-  const int tg = token_group_for(batch);
+  const size_t smem = moe::mma_smem_bytes(h->n_stages);
 
   auto bail = [&](cudaError_t err) {
     h->dirty = true;
@@ -238,56 +341,42 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     return h->timing ? cudaEventRecord(h->tev[i], st) : cudaSuccess;
   };
 
-  if (s.n_shared) {
-    if (fork) {
-      if ((e = cudaEventRecord(h->ev_fork, sm)) != cudaSuccess) return bail(e);
-      if ((e = cudaStreamWaitEvent(sa, h->ev_fork, 0)) != cudaSuccess) return bail(e);
-    }
-    GemvArgs ga{};
-    ga.dense_w = static_cast<const __nv_bfloat16*>(shared_w13);
-    ga.K = h->sh_up.K;
-    ga.N = h->sh_up.N;
-    ga.I = h->sh_up.I;
-    ga.panel_w = h->sh_up.panel_w;
-    ga.n_cp = h->sh_up.n_cp;
-    ga.stage_rows = h->sh_up.stage_rows;
+  // Shared expert (weight 1, all tokens): on stream_aux, forked after the
+  // router is enqueued so the router's CTAs are dispatched first.  Its grid
+  // is sized to its share of the bytes (the rest of the SMs stream routed
+  // experts), so both finish together instead of contending for every SM.
+  auto launch_shared = [&](cudaStream_t st_sh) -> cudaError_t {
+    MmaArgs ga{};
+    ga.H = s.hidden;
+    ga.I = s.shared_inter;
+    ga.panel_stride = moe::max_up_panels(s.shared_inter);
     ga.n_stages = h->n_stages;
     ga.batch = batch;
     ga.max_units = 1;
+    ga.w13 = static_cast<const __nv_bfloat16*>(shared_w13);
+    ga.w2 = static_cast<const __nv_bfloat16*>(shared_w2);
+    ga.maps13 = maps + 2 * (size_t)s.n_experts * mb;
+    ga.maps2 = maps + (2 * (size_t)s.n_experts + 1) * mb;
     ga.plan = nullptr;
     ga.x = static_cast<const __nv_bfloat16*>(x);
     ga.h = h->at<float>(h->L.h_s);
-    ga.a_out = h->at<float>(h->L.a_s);
-    ga.counters = h->at<unsigned>(h->L.counters_s);
+    ga.a = h->at<__nv_bfloat16>(h->L.a_s);
+    ga.acc = acc;
+    ga.panel_cnt = h->at<unsigned>(h->L.panel_cnt_s);
+    ga.panel_ready = h->at<unsigned>(h->L.panel_ready_s);
+    ga.queue = h->at<unsigned>(h->L.queue_s);
     ga.status = status;
-    const size_t smem = moe::gemv_smem_bytes(h->n_stages, tg);
-    const cudaStream_t st_sh = fork ? sa : sm;
-    if ((e = mark(5, st_sh)) != cudaSuccess) return bail(e);
-    e = launch(pick_gemv<true, true>(tg), h->grid_shared, moe::kGemvThreads, smem, st_sh, false, ga, *h->tab13);
-    if (e != cudaSuccess) return bail(e);
+    cudaError_t err = mark(4, st_sh);
+    if (err != cudaSuccess) return err;
+    err = launch(pick_mlp<true>(moe::class_for_tokens(batch), h->use_tmap), shared_grid(h, batch), moe::kGemvThreads, smem,
+                 st_sh, false, ga, *h->tab_none, *h->tab_none);
+    if (err != cudaSuccess) return err;
     ++kernels;
-    if ((e = mark(6, st_sh)) != cudaSuccess) return bail(e);
-    GemvArgs gd{};
-    gd.dense_w = static_cast<const __nv_bfloat16*>(shared_w2);
-    gd.K = h->sh_down.K;
-    gd.N = h->sh_down.N;
-    gd.I = 0;
-    gd.panel_w = h->sh_down.panel_w;
-    gd.n_cp = h->sh_down.n_cp;
-    gd.stage_rows = h->sh_down.stage_rows;
-    gd.n_stages = h->n_stages;
-    gd.batch = batch;
-    gd.max_units = 1;
-    gd.a_in = h->at<float>(h->L.a_s);
-    gd.acc = acc;
-    gd.status = status;
-    e = launch(pick_gemv<true, false>(tg), h->grid_shared, moe::kGemvThreads, smem, st_sh, true, gd, *h->tab2);
-    if (e != cudaSuccess) return bail(e);
-    ++kernels;
-    if ((e = mark(7, st_sh)) != cudaSuccess) return bail(e);
-    if (fork) {
-      if ((e = cudaEventRecord(h->ev_join, sa)) != cudaSuccess) return bail(e);
-    }
+    return mark(5, st_sh);
+  };
+  if (fork) {
+    if ((e = cudaEventRecord(h->ev_fork, sm)) != cudaSuccess) return bail(e);
+    if ((e = cudaStreamWaitEvent(sa, h->ev_fork, 0)) != cudaSuccess) return bail(e);
   }
 
   // Router + top-k + plan.
@@ -313,47 +402,45 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   if (e != cudaSuccess) return bail(e);
   ++kernels;
   if ((e = mark(1, sm)) != cudaSuccess) return bail(e);
+  if (fork) {
+    if ((e = launch_shared(sa)) != cudaSuccess) return bail(e);
+    if ((e = cudaEventRecord(h->ev_join, sa)) != cudaSuccess) return bail(e);
+  }
 
-  const size_t smem = moe::gemv_smem_bytes(h->n_stages, tg);
-  GemvArgs ua{};
-  ua.K = h->up.K;
-  ua.N = h->up.N;
-  ua.I = h->up.I;
-  ua.panel_w = h->up.panel_w;
-  ua.n_cp = h->up.n_cp;
-  ua.stage_rows = h->up.stage_rows;
-  ua.n_stages = h->n_stages;
-  ua.batch = batch;
-  ua.max_units = s.n_experts;
-  ua.plan = h->at<Plan>(h->L.plan);
-  ua.x = static_cast<const __nv_bfloat16*>(x);
-  ua.h = h->at<float>(h->L.h);
-  ua.a_out = h->at<float>(h->L.a);
-  ua.counters = h->at<unsigned>(h->L.counters);
-  ua.status = status;
-  e = launch(pick_gemv<false, true>(tg), h->grid_routed, moe::kGemvThreads, smem, sm, true, ua, *h->tab13);
+  // Routed experts: UP + SwiGLU + DOWN in one persistent launch.
+  MmaArgs ma{};
+  ma.H = s.hidden;
+  ma.I = s.inter;
+  ma.panel_stride = moe::max_up_panels(s.inter);
+  ma.n_stages = h->n_stages;
+  ma.batch = batch;
+  ma.max_units = (int)max_units(&s);
+  ma.plan = h->at<Plan>(h->L.plan);
+  ma.maps13 = maps;
+  ma.maps2 = maps + (size_t)s.n_experts * mb;
+  ma.x = static_cast<const __nv_bfloat16*>(x);
+  ma.h = h->at<float>(h->L.h);
+  ma.a = h->at<__nv_bfloat16>(h->L.a);
+  ma.acc = acc;
+  ma.panel_cnt = h->at<unsigned>(h->L.panel_cnt);
+  ma.panel_ready = h->at<unsigned>(h->L.panel_ready);
+  ma.queue = h->at<unsigned>(h->L.queue);
+  ma.status = status;
+  int g_routed = h->grid_routed;
+  if (fork && h->grid_routed_auto) {
+    g_routed = h->num_sms - shared_grid(h, batch);
+    if (g_routed < 1) g_routed = 1;
+  }
+  // a unit holds at most kMaxUnitTokens tokens (larger experts are split)
+  const int routed_kc = moe::class_for_tokens(batch < moe::kMaxUnitTokens ? batch : moe::kMaxUnitTokens);
+  e = launch(pick_mlp<false>(routed_kc, h->use_tmap), g_routed, moe::kGemvThreads, smem, sm, true, ma, *h->tab13,
+             *h->tab2);
   if (e != cudaSuccess) return bail(e);
   ++kernels;
   if ((e = mark(2, sm)) != cudaSuccess) return bail(e);
-
-  GemvArgs da{};
-  da.K = h->down.K;
-  da.N = h->down.N;
-  da.I = 0;
-  da.panel_w = h->down.panel_w;
-  da.n_cp = h->down.n_cp;
-  da.stage_rows = h->down.stage_rows;
-  da.n_stages = h->n_stages;
-  da.batch = batch;
-  da.max_units = s.n_experts;
-  da.plan = h->at<Plan>(h->L.plan);
-  da.a_in = h->at<float>(h->L.a);
-  da.acc = acc;
-  da.status = status;
-  e = launch(pick_gemv<false, false>(tg), h->grid_routed, moe::kGemvThreads, smem, sm, true, da, *h->tab2);
-  if (e != cudaSuccess) return bail(e);
-  ++kernels;
-  if ((e = mark(3, sm)) != cudaSuccess) return bail(e);
+  if (s.n_shared && !fork) {
+    if ((e = launch_shared(sm)) != cudaSuccess) return bail(e);
+  }
 
   if (fork) {
     if ((e = cudaStreamWaitEvent(sm, h->ev_join, 0)) != cudaSuccess) return bail(e);
@@ -363,13 +450,12 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
              static_cast<const __nv_bfloat16*>(x), acc, static_cast<__nv_bfloat16*>(out), nvec);
   if (e != cudaSuccess) return bail(e);
   ++kernels;
-  if ((e = mark(4, sm)) != cudaSuccess) return bail(e);
+  if ((e = mark(3, sm)) != cudaSuccess) return bail(e);
 
   h->stats.forwards += 1;
   h->stats.kernels_launched += (uint64_t)kernels;
   h->stats.last_kernels = kernels;
-  h->stats.last_variant = tg;
-  h->stats.variant_calls[tg == 1 ? 0 : (tg == 2 ? 1 : (tg == 4 ? 2 : 3))] += 1;
+  h->stats.last_token_tiles = ((batch < moe::kMaxUnitTokens ? batch : moe::kMaxUnitTokens) + 7) / 8;
   return MOE_OK;
 }
 
@@ -563,9 +649,11 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
   h->s = *shapes;
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
-  h->n_stages = env_int("MOE_DECODE_STAGES", 6, 2, moe::kMaxStages);
-  h->grid_routed = env_int("MOE_DECODE_GRID_ROUTED", h->num_sms, 1, 8 * h->num_sms);
-  h->grid_shared = env_int("MOE_DECODE_GRID_SHARED", h->num_sms, 1, 8 * h->num_sms);
+  h->n_stages = env_int("MOE_DECODE_STAGES", 3, 2, moe::kMaxStagesMma);
+  h->grid_routed = env_int("MOE_DECODE_GRID_ROUTED", 0, 0, 8 * h->num_sms);
+  h->grid_routed_auto = h->grid_routed == 0;
+  if (h->grid_routed == 0) h->grid_routed = h->num_sms;
+  h->grid_shared = env_int("MOE_DECODE_GRID_SHARED", 0, 0, 8 * h->num_sms);  // 0: sized per call
   {
     int gr = h->num_sms;
     const int cap = shapes->hidden / 8;
@@ -576,18 +664,14 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
     h->router_chunk_rows = rows < cap_rows ? rows : cap_rows;
     if (h->router_chunk_rows < 1) h->router_chunk_rows = 1;
   }
-  h->up = make_geom(true, shapes->hidden, shapes->inter);
-  h->down = make_geom(false, shapes->inter, shapes->hidden);
-  if (shapes->n_shared) {
-    h->sh_up = make_geom(true, shapes->hidden, shapes->shared_inter);
-    h->sh_down = make_geom(false, shapes->shared_inter, shapes->hidden);
-  }
   h->L = layout_for(shapes);
   h->tab13 = new (std::nothrow) ExpertTable();
   h->tab2 = new (std::nothrow) ExpertTable();
-  if (!h->tab13 || !h->tab2) {
+  h->tab_none = new (std::nothrow) ExpertTable();
+  if (!h->tab13 || !h->tab2 || !h->tab_none) {
     delete h->tab13;
     delete h->tab2;
+    delete h->tab_none;
     delete h;
     return MOE_ERR_OUT_OF_MEMORY;
   }
@@ -603,6 +687,22 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
     rc = fail_cuda(e);
   if (rc == MOE_OK && (e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming)) != cudaSuccess)
     rc = fail_cuda(e);
+  if (rc == MOE_OK && (e = cudaEventCreateWithFlags(&h->ev_maps, cudaEventDisableTiming)) != cudaSuccess)
+    rc = fail_cuda(e);
+  if (rc == MOE_OK) {
+    // tensor-map path: shapes in whole 64-column chunks and a working encoder
+    const bool shapes_ok = shapes->hidden % moe::kChunkCols == 0 && shapes->inter % moe::kChunkCols == 0 &&
+                           (!shapes->n_shared || shapes->shared_inter % moe::kChunkCols == 0);
+    uint8_t probe[moe::kTensorMapBytes];
+    h->use_tmap = env_int("MOE_DECODE_TMAP", 1, 0, 1) == 1 && shapes_ok &&
+                  encode_matrix_map(probe, h->ws, shapes->hidden, 2 * shapes->inter);
+    if (h->use_tmap) {
+      h->map_ptrs.assign(2 * (size_t)shapes->n_experts + 2, nullptr);
+      e = cudaMallocHost(reinterpret_cast<void**>(&h->maps_host),
+                         (2 * (size_t)shapes->n_experts + 2) * moe::kTensorMapBytes);
+      if (e != cudaSuccess) rc = fail_cuda(e);
+    }
+  }
   if (rc == MOE_OK) rc = set_kernel_attrs(h);
   if (rc != MOE_OK) {
     moe_decode_destroy(h);
@@ -665,9 +765,12 @@ int moe_decode_destroy(moe_decode_t h) {
     }
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->ev_maps) cudaEventDestroy(h->ev_maps);
+    if (h->maps_host) cudaFreeHost(h->maps_host);
   }
   delete h->tab13;
   delete h->tab2;
+  delete h->tab_none;
   delete h;
   return rc;
 }

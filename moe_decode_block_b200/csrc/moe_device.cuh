@@ -14,10 +14,16 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kMaxBatch = 64;
 constexpr int kMaxAssign = kMaxBatch * kMaxTopK;
+// A unit is one pass of the expert kernels over one expert's weights; an
+// expert routed more than kMaxUnitTokens tokens is split into several units.
+constexpr int kMaxUnitTokens = 32;
+constexpr int kMaxUnits = kMaxExperts + kMaxAssign / kMaxUnitTokens;
 
-// Expert GEMV kernels: 16 consumer warps own one 16-byte column vector each
-// (8 bf16 columns), one producer warp issues the TMA bulk copies.
-constexpr int kConsumerWarps = 16;
+// Expert kernels: 8 consumer warps split a panel's columns; one producer warp
+// issues the TMA loads.  Nine warps per CTA leave each thread up to 168
+// registers (a 17-warp CTA would cap them at 96), enough for 128 fp32
+// accumulators without spilling.
+constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kGemvThreads = kConsumerThreads + 32;
 constexpr int kMaxPanelCols = 8 * kConsumerThreads;  // local columns per panel
@@ -37,14 +43,16 @@ constexpr int kStatusPlan = 2;
 constexpr uint32_t kSpinLimit = 1u << 24;
 
 // Routing plan: written by the last router CTA, read by the expert kernels.
-// Units are the active experts in ascending id order; the assignments of
-// unit u are [unit_begin[u], unit_begin[u] + unit_count[u]) sorted by token.
+// Units follow the active experts in ascending id order (an expert with more
+// than kMaxUnitTokens tokens gets several consecutive units); the
+// assignments of unit u are [unit_begin[u], unit_begin[u] + unit_count[u]),
+// sorted by token.
 struct Plan {
-  int n_active;
+  int n_active;  // number of units
   int pad_[3];
-  int unit_expert[kMaxExperts];
-  int unit_begin[kMaxExperts];
-  int unit_count[kMaxExperts];
+  int unit_expert[kMaxUnits];
+  int unit_begin[kMaxUnits];
+  int unit_count[kMaxUnits];
   int assign_tok[kMaxAssign];   // token index b
   int assign_slot[kMaxAssign];  // b * top_k + j (row of the per-assignment buffers)
   float assign_w[kMaxAssign];   // renormalised routing weight
@@ -131,6 +139,27 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+// Same without a cache hint (activations: small and re-read by many CTAs).
+__device__ __forceinline__ void bulk_copy_g2s_plain(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// TMA tiled load of a 3-D box described by a tensor map in global memory
+// (no multicast), completion counted on `bar`.  dst must be 1024-byte
+// aligned when the map uses 128-byte swizzling.
+__device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, int c1, int c2, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+      "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar)), "l"(policy)
       : "memory");
 }
 

@@ -240,13 +240,14 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   for (int i = tid; i < nas; i += kRouterThreads) atomicAdd(&s_cnt[s_ids[i]], 1);
   __syncthreads();
 
-  // Exclusive scans of counts and of active flags over E (<= 1024 = 4/thread).
+  // Exclusive scans of counts and of units per expert over E (<= 1024 =
+  // 4/thread); an expert with c tokens gets ceil(c / kMaxUnitTokens) units.
   int c4[4], f4[4], csum = 0, fsum = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int e = tid * 4 + i;
     c4[i] = e < E ? s_cnt[e] : 0;
-    f4[i] = c4[i] > 0 ? 1 : 0;
+    f4[i] = (c4[i] + kMaxUnitTokens - 1) / kMaxUnitTokens;
     csum += c4[i];
     fsum += f4[i];
   }
@@ -259,10 +260,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
     if (e < E) {
       s_off[e] = cbase;
       s_act[e] = f4[i] ? fbase : -1;
-      if (f4[i]) {
-        a.plan->unit_expert[fbase] = e;
-        a.plan->unit_begin[fbase] = cbase;
-        a.plan->unit_count[fbase] = c4[i];
+      for (int j = 0; j < f4[i]; ++j) {
+        a.plan->unit_expert[fbase + j] = e;
+        a.plan->unit_begin[fbase + j] = cbase + j * kMaxUnitTokens;
+        a.plan->unit_count[fbase + j] = min(kMaxUnitTokens, c4[i] - j * kMaxUnitTokens);
       }
     }
     cbase += c4[i];

@@ -45,6 +45,9 @@ class BlockShape:
 
 TINY = BlockShape(hidden=256, n_experts=16, top_k=2, inter=128, shared_inter=128)
 FULL = BlockShape(hidden=7168, n_experts=384, top_k=8, inter=2048, shared_inter=2048)
+# Same per-expert shapes as FULL with only 16 experts (1.4 GB of weights):
+# the small case used for detailed profiler captures.
+PROF = BlockShape(hidden=7168, n_experts=16, top_k=8, inter=2048, shared_inter=2048)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -65,6 +68,10 @@ WORKLOADS: Dict[str, Workload] = {
     "full_b64": Workload("full_b64", FULL, 64, "uniform", "full-size block, batch 64, uniform-ish routing"),
     "zipf_b32": Workload("zipf_b32", FULL, 32, "zipf",
                          "full-size block, batch 32, Zipf(1.2) per-expert log-prior added to router logits"),
+    "prof_b1": Workload("prof_b1", PROF, 1, "uniform",
+                        "profiling case: full-size experts, 16 of them (1.4 GB), batch 1"),
+    "prof_b8": Workload("prof_b8", PROF, 8, "uniform",
+                        "profiling case: full-size experts, 16 of them (1.4 GB), batch 8"),
 }
 
 
