@@ -76,11 +76,19 @@ constexpr int kNumClasses = 4;
 __host__ __device__ constexpr int class_lw(int c) { return c <= 1 ? 2048 : (c == 2 ? 1024 : 512); }
 __host__ __device__ constexpr int class_rows(int c) { return c <= 1 ? 16 : (c == 2 ? 32 : 64); }
 __host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : (c == 2 ? 4 : 8)); }
-__host__ __device__ constexpr int class_mt(int c) { return class_lw(c) / (kConsumerWarps * 16); }
 __host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : (n <= 32 ? 2 : 3)); }
+// Consumer warps of the instance compiled for classes <= kc: sixteen when a
+// thread needs only 32 accumulators (more warps hide more latency), eight
+// otherwise -- nine warps per CTA leave each thread 168 registers, enough for
+// 128 accumulators, where seventeen warps cap it at 96.
+__host__ __device__ constexpr int consumer_warps_for(int kc) { return kc == 0 ? 16 : 8; }
+__host__ __device__ constexpr int expert_threads(int kc) { return (consumer_warps_for(kc) + 1) * 32; }
+// m-tiles (16 columns) per consumer warp for class c with cw consumer warps
+__host__ __device__ constexpr int class_mt(int c, int cw) { return class_lw(c) / (cw * 16); }
 // accumulator fragments (of 4 floats) a consumer thread needs for classes <= KC
 __host__ __device__ constexpr int acc_frags(int kc) {
-  return kc == 0 ? class_mt(0) * class_nt(0) : class_mt(1) * class_nt(1);
+  return kc == 0 ? class_mt(0, consumer_warps_for(0)) * class_nt(0)
+                 : class_mt(1, consumer_warps_for(kc)) * class_nt(1);
 }
 constexpr int kStageWBytes = 65536 + 64 * 16;              // rows * (2*LW + 16), largest over classes
 constexpr int kStageXBytes = kMaxTok * (64 * 2 + 16);      // tokens * (2*rows + 16), largest
@@ -175,11 +183,11 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
 
 // One stage of tensor-core work for class C: this warp's MT m-tiles against
 // the stage's token tiles, accumulated into acc[mt * NT + nt][0..3].
-template <int C, int NF, bool TMAP>
+template <int C, int NF, bool TMAP, int CW>
 __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint32_t sx, int LW, int nrows,
                                           int ntiles, int warp, int lane) {
   constexpr int LWc = class_lw(C), R = class_rows(C);
-  constexpr int MT = class_mt(C), NT = class_nt(C), KS = R / 16;
+  constexpr int MT = class_mt(C, CW), NT = class_nt(C), KS = R / 16;
   static_assert(MT * NT <= NF, "accumulator budget");
   constexpr int pitch = LWc * 2 + 16, xpitch = R * 2 + 16;
   constexpr int rbstride = (LWc / kChunkCols) * kChunkTile;  // tensor-map layout: one 16-row block
@@ -241,37 +249,62 @@ __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint
 
 // Flush this warp's partial sums of a piece (class C) with fp32 atomics.
 // Local columns: DOWN [0, w) -> c0 + l; UP gate [0, w) -> c0 + l and up
-// [uoff, uoff + w) -> I + c0 + (l - uoff); anything else is padding.
-template <int C, int NF>
+// [uoff, uoff + w) -> I + c0 + (l - uoff); anything else is padding.  w and
+// uoff are multiples of 8, so four consecutive local columns map to four
+// consecutive output columns.
+__device__ __forceinline__ int local_to_col(int l, bool up, int c0, int w, int uoff, int I) {
+  if (!up) return l < w ? c0 + l : -1;
+  if (l < w) return c0 + l;
+  if (l >= uoff && l < uoff + w) return I + c0 + (l - uoff);
+  return -1;
+}
+
+// Flush this warp's partial sums of a piece (class C) with fp32 atomics.  An
+// m-tile's C fragment spreads 16 columns of a token over 8 lanes; shuffles
+// gather each run of 4 columns into one lane, so every 16 bytes take one
+// vector atomic instead of four scalar ones.
+template <int C, int NF, int CW>
 __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], const MmaArgs& args, const StageHdr& hd,
                                             bool up, int c0, int w, int uoff, int LW, int warp, int lane) {
-  constexpr int MT = class_mt(C), NT = class_nt(C);
+  constexpr int MT = class_mt(C, CW), NT = class_nt(C);
   const int m0 = warp * MT * 16;
   if (m0 >= LW) return;
   const int gid = lane >> 2, tig = lane & 3;
   const int I = args.I, H = args.H;
+  const int ntiles = (hd.ntok + 7) >> 3;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
+    if (nt >= ntiles) break;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int n = nt * 8 + tig * 2 + e;
-      if (n >= hd.ntok) continue;
-      const int r = hd.row[n];
-      const float wt = up ? 1.f : hd.wt[n];
-      float* row = up ? args.h + (size_t)r * (2 * I) : args.acc + (size_t)r * H;
+      const int n = nt * 8 + tig * 2 + e;  // this lane's token (same for its tig group)
+      const bool valid = n < hd.ntok;
+      float* row = nullptr;
+      float wt = 1.f;
+      if (valid) {
+        const int r = hd.row[n];
+        wt = up ? 1.f : hd.wt[n];
+        row = up ? args.h + (size_t)r * (2 * I) : args.acc + (size_t)r * H;
+      }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
+        if (m0 + mt * 16 >= LW) break;
+        const float v_lo = acc[mt * NT + nt][e];      // column gid
+        const float v_hi = acc[mt * NT + nt][2 + e];  // column gid + 8
+        // lane with gid < 4 collects columns 4*gid .. 4*gid + 3 of its token
+        float o[4];
 #pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-          const int l = m0 + mt * 16 + gid + hi * 8;  // local column
-          int col = -1;
-          if (!up)
-            col = l < w ? c0 + l : -1;
-          else if (l < w)
-            col = c0 + l;
-          else if (l >= uoff && l < uoff + w)
-            col = I + c0 + (l - uoff);
-          if (col >= 0) atomicAdd(row + col, wt * acc[mt * NT + nt][hi * 2 + e]);
+        for (int j = 0; j < 4; ++j) {
+          const int c = 4 * (gid & 3) + j;
+          const int src = ((c & 7) << 2) | tig;
+          const float a = __shfl_sync(0xffffffffu, v_lo, src);
+          const float b = __shfl_sync(0xffffffffu, v_hi, src);
+          o[j] = c < 8 ? a : b;
+        }
+        if (valid && gid < 4) {
+          const int col = local_to_col(m0 + mt * 16 + 4 * gid, up, c0, w, uoff, I);
+          if (col >= 0)
+            atomicAdd(reinterpret_cast<float4*>(row + col), make_float4(wt * o[0], wt * o[1], wt * o[2], wt * o[3]));
         }
       }
     }
@@ -279,7 +312,7 @@ __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], const Mma
 }
 
 template <bool DENSE, int KC, bool TMAP>
-__global__ void __launch_bounds__(kGemvThreads, 1)
+__global__ void __launch_bounds__(expert_threads(KC), 1)
     expert_mlp_kernel(const __grid_constant__ MmaArgs args, const __grid_constant__ ExpertTable tab13,
                       const __grid_constant__ ExpertTable tab2) {
   extern __shared__ __align__(1024) uint8_t mma_smem[];
@@ -292,13 +325,14 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
   volatile int* s_misc = reinterpret_cast<volatile int*>(hdr + kMaxStagesMma);
   // s_misc[0]: abort flag (a bounded wait gave up), [2]: stages issued
 
+  constexpr int CW = consumer_warps_for(KC);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool is_producer = (warp == kConsumerWarps);
+  const bool is_producer = (warp == CW);
 
   if (tid == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(&full[i], 1);
-      mbar_init(&empty[i], kConsumerWarps);
+      mbar_init(&empty[i], CW);
     }
     s_misc[0] = 0;
     s_misc[2] = 0;
@@ -335,9 +369,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     };
     auto unit_stages = [&](int u, bool up) {
       const int c = unit_class(unit_tokens(u));
-      return (long long)unit_panels(c, up, H, I) * unit_panel_stages(c, up, H, I);
+      return unit_panels(c, up, H, I) * unit_panel_stages(c, up, H, I);
     };
-    long long T_up = 0, T_dn = 0;
+    int T_up = 0, T_dn = 0;  // at most ~1.5M stages: 32-bit arithmetic
     for (int u = lane; u < n_units; u += 32) {
       T_up += unit_stages(u, true);
       T_dn += unit_stages(u, false);
@@ -347,19 +381,29 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       T_up += __shfl_xor_sync(0xffffffffu, T_up, off);
       T_dn += __shfl_xor_sync(0xffffffffu, T_dn, off);
     }
-    const long long T_all = T_up + T_dn;
-    const long long G = gridDim.x;
-    long long c_big = T_all / (4 * G);
+    const int T_all = T_up + T_dn;
+    const int G = gridDim.x;
+    // ticket -> range: 3/4 of the list in chunks of c_big, then 3/16 in
+    // chunks of c_big / 4, then single stages
+    int c_big = T_all / (4 * G);
     c_big = c_big < 1 ? 1 : (c_big > kMaxChunk ? kMaxChunk : c_big);
-    const long long n_big = (T_all * 3 / 4) / c_big;
-    auto chunk_of = [&](long long tk, long long& b, long long& e) {
+    const int c_mid = c_big / 4 < 1 ? 1 : c_big / 4;
+    const int n_big = (T_all / 4 * 3) / c_big;
+    const int T1 = n_big * c_big;
+    const int n_mid = ((T_all - T1) / 4 * 3) / c_mid;
+    const int T2 = T1 + n_mid * c_mid;
+    auto chunk_of = [&](int tk, int& b, int& e) {
       if (tk < n_big) {
         b = tk * c_big;
         e = b + c_big;
+      } else if (tk - n_big < n_mid) {
+        b = T1 + (tk - n_big) * c_mid;
+        e = b + c_mid;
       } else {
-        b = n_big * c_big + (tk - n_big);
+        b = T2 + (tk - n_big - n_mid);
         e = b + 1;
       }
+      if (b > T_all) b = T_all;
       if (e > T_all) e = T_all;
     };
     // cursor over the work list (tickets only grow, so it only moves forward).
@@ -370,7 +414,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     // go to L2 every time.
     bool cur_up = true;
     int cur_unit = 0;
-    long long cur_base = 0, cur_size = n_units > 0 ? unit_stages(0, true) : 0;
+    int cur_base = 0, cur_size = n_units > 0 ? unit_stages(0, true) : 0;
     int u_loaded = -1;
     bool u_loaded_up = true;
     int u_ntok = 0, u_cls = 0, u_lw = 0, u_R = 0, u_S = 0, u_begin = 0, u_row0 = 0, u_row1 = 0;
@@ -380,18 +424,18 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
     const uint8_t* u_map = nullptr;
     uint32_t q = 0;
     int ready_panel = -1;  // last (unit, UP panel) seen published
-    long long tk = 0;
-    if (lane == 0) tk = (long long)atomicAdd(&args.queue[0], 1u);
+    int tk = 0;
+    if (lane == 0) tk = (int)atomicAdd(&args.queue[0], 1u);
     tk = __shfl_sync(0xffffffffu, tk, 0);
     while (true) {
-      long long c_beg, c_end;
+      int c_beg, c_end;
       chunk_of(tk, c_beg, c_end);
       if (c_beg >= T_all || *abort_flag) break;
-      long long tk_next = 0;  // next ticket now: its latency overlaps this chunk
-      if (lane == 0) tk_next = (long long)atomicAdd(&args.queue[0], 1u);
-      long long piece_start = c_beg;
+      int tk_next = 0;  // next ticket now: its latency overlaps this chunk
+      if (lane == 0) tk_next = (int)atomicAdd(&args.queue[0], 1u);
+      int piece_start = c_beg;
       bool stop = false;
-      for (long long t = c_beg; t < c_end; ++t, ++q) {
+      for (int t = c_beg; t < c_end; ++t, ++q) {
         while (t >= cur_base + cur_size) {
           cur_base += cur_size;
           if (++cur_unit == n_units) {
@@ -435,9 +479,9 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           }
         }
         const int ntok = u_ntok, cls = u_cls, lw = u_lw, R = u_R, S = u_S, begin = u_begin;
-        const long long loc = t - cur_base;
-        const int cp = (int)(loc / S);
-        const int st = (int)(loc - (long long)cp * S);
+        const int loc = t - cur_base;
+        const int cp = loc / S;
+        const int st = loc - cp * S;
         if (t == c_beg || st == 0) piece_start = t;
         const bool first = (t == piece_start);
         const bool last = (t == c_end - 1 || st == S - 1);
@@ -509,7 +553,7 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
           hd.flags = (first ? kFirst : 0) | (last ? kLast : 0);
           hd.ntok = ntok;
           hd.begin = begin;
-          hd.pstages = (int)(t - piece_start + 1);
+          hd.pstages = t - piece_start + 1;
         }
         __syncwarp();  // every lane's header writes precede lane 0's (releasing) arrive
         if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
@@ -607,42 +651,42 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
       const uint32_t sw = smem_addr(stages + (size_t)slot * kStageBytesMma);
       const uint32_t sx = sw + kStageWBytes;
       if (hd.cls == 0)
-        mma_stage<0, NF, TMAP>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+        mma_stage<0, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
       else if constexpr (KC >= 1) {
         if (hd.cls == 1)
-          mma_stage<1, NF, TMAP>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+          mma_stage<1, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
         else if constexpr (KC >= 2) {
           if (hd.cls == 2)
-            mma_stage<2, NF, TMAP>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+            mma_stage<2, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
           else if constexpr (KC >= 3)
-            mma_stage<3, NF, TMAP>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+            mma_stage<3, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
         }
       }
       if (hd.flags & kLast) {
         // ------------------------------------------- flush the piece's sums
         if (!*abort_flag) {
           if (hd.cls == 0)
-            flush_piece<0, NF>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
+            flush_piece<0, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
           else if constexpr (KC >= 1) {
             if (hd.cls == 1)
-              flush_piece<1, NF>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
+              flush_piece<1, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
             else if constexpr (KC >= 2) {
               if (hd.cls == 2)
-                flush_piece<2, NF>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
+                flush_piece<2, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
               else if constexpr (KC >= 3)
-                flush_piece<3, NF>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
+                flush_piece<3, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
             }
           }
         }
         if (up) {
           // ---------------- last warp to finish a panel applies the SwiGLU.
           // Every consumer warp counts its own stages of the piece, so the
-          // panel is complete when its counter reaches (stages * 16); no
+          // panel is complete when its counter reaches (stages * CW); no
           // barrier across warps is needed.
           __threadfence();
           __syncwarp();
           const int panel = hd.unit * args.panel_stride + hd.cp;
-          const unsigned target = (unsigned)unit_panel_stages(hd.cls, true, H, I) * kConsumerWarps;
+          const unsigned target = (unsigned)unit_panel_stages(hd.cls, true, H, I) * CW;
           int last = 0;
           if (lane == 0 && !*abort_flag) {
             const unsigned steps = (unsigned)hd.pstages;

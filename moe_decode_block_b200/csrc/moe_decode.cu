@@ -368,7 +368,8 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     ga.status = status;
     cudaError_t err = mark(4, st_sh);
     if (err != cudaSuccess) return err;
-    err = launch(pick_mlp<true>(moe::class_for_tokens(batch), h->use_tmap), shared_grid(h, batch), moe::kGemvThreads, smem,
+    const int kc_s = moe::class_for_tokens(batch);
+    err = launch(pick_mlp<true>(kc_s, h->use_tmap), shared_grid(h, batch), moe::expert_threads(kc_s), smem,
                  st_sh, false, ga, *h->tab_none, *h->tab_none);
     if (err != cudaSuccess) return err;
     ++kernels;
@@ -433,7 +434,8 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   }
   // a unit holds at most kMaxUnitTokens tokens (larger experts are split)
   const int routed_kc = moe::class_for_tokens(batch < moe::kMaxUnitTokens ? batch : moe::kMaxUnitTokens);
-  e = launch(pick_mlp<false>(routed_kc, h->use_tmap), g_routed, moe::kGemvThreads, smem, sm, true, ma, *h->tab13,
+  e = launch(pick_mlp<false>(routed_kc, h->use_tmap), g_routed, moe::expert_threads(routed_kc), smem, sm, true, ma,
+             *h->tab13,
              *h->tab2);
   if (e != cudaSuccess) return bail(e);
   ++kernels;

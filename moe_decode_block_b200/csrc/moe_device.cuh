@@ -19,17 +19,6 @@ constexpr int kMaxAssign = kMaxBatch * kMaxTopK;
 constexpr int kMaxUnitTokens = 32;
 constexpr int kMaxUnits = kMaxExperts + kMaxAssign / kMaxUnitTokens;
 
-// Expert kernels: 8 consumer warps split a panel's columns; one producer warp
-// issues the TMA loads.  Nine warps per CTA leave each thread up to 168
-// registers (a 17-warp CTA would cap them at 96), enough for 128 fp32
-// accumulators without spilling.
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kGemvThreads = kConsumerThreads + 32;
-constexpr int kMaxPanelCols = 8 * kConsumerThreads;  // local columns per panel
-constexpr int kStepRows = 64;    // rows per partition step (and per activation chunk)
-constexpr int kStageBytes = 32 * 1024;
-constexpr int kMaxStages = 8;
 
 constexpr int kRouterThreads = 256;
 
@@ -166,11 +155,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, 
 // Bulk prefetch of a global range into L2 (no data returned to the SM).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// Named barrier over the consumer warps only (the producer warp never joins).
-__device__ __forceinline__ void consumer_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads) : "memory");
 }
 
 __device__ __forceinline__ void bf16x2_to_f32(uint32_t v, float& lo, float& hi) {
