@@ -349,6 +349,12 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   if (is_producer) {
     // ================================================================ producer
     const uint64_t pol = l2_evict_first_policy();
+    // The first ticket only touches this kernel's own counter (returned to
+    // zero by the previous launch of this kernel, which finished before the
+    // router started), so take it before the wait: its round trip overlaps
+    // the router's tail.  It is turned into a range only after the wait.
+    int tk = 0;
+    if (lane == 0) tk = (int)atomicAdd(&args.queue[0], 1u);
     cudaGridDependencySynchronize();  // the plan and the activations come from earlier kernels
     const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
     int n_units = 1;
@@ -424,8 +430,6 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
     const uint8_t* u_map = nullptr;
     uint32_t q = 0;
     int ready_panel = -1;  // last (unit, UP panel) seen published
-    int tk = 0;
-    if (lane == 0) tk = (int)atomicAdd(&args.queue[0], 1u);
     tk = __shfl_sync(0xffffffffu, tk, 0);
     while (true) {
       int c_beg, c_end;

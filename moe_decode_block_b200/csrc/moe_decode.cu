@@ -223,14 +223,17 @@ struct moe_decode_ctx {
 
 namespace {
 
-int router_grid(const moe_decode_ctx* h, int batch) {
-  int g = h->grid_router_max;
-  if (batch > 8) {
-    const int cap = h->num_sms * 8 / batch;
-    g = g < cap ? g : cap;
-  }
-  if (g < 1) g = 1;
-  return g;
+int router_grid(const moe_decode_ctx* h, int /*batch*/) {
+  return h->grid_router_max < 1 ? 1 : h->grid_router_max;
+}
+
+// Router kernel holding E <= 32 * NV logits per lane during top-k.
+using RouterKernel = void (*)(RouterArgs);
+RouterKernel pick_router(int n_experts) {
+  if (n_experts <= 128) return moe::router_topk_kernel<4>;
+  if (n_experts <= 256) return moe::router_topk_kernel<8>;
+  if (n_experts <= 512) return moe::router_topk_kernel<16>;
+  return moe::router_topk_kernel<32>;
 }
 
 // CTAs for the shared expert when it runs beside the routed experts: its
@@ -266,7 +269,7 @@ int set_kernel_attrs(const moe_decode_ctx* h) {
     }
   }
   const int rsmem = (int)moe::router_smem_bytes(h->s.max_batch, h->s.n_experts, h->router_chunk_rows);
-  e = cudaFuncSetAttribute(moe::router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
+  e = cudaFuncSetAttribute(pick_router(h->s.n_experts), cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
   if (e != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }
@@ -398,7 +401,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   ra.topk_w = topk_w;
   ra.status = status;
   if ((e = mark(0, sm)) != cudaSuccess) return bail(e);
-  e = launch(moe::router_topk_kernel, ra.G, moe::kRouterThreads,
+  e = launch(pick_router(s.n_experts), ra.G, moe::kRouterThreads,
              moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra);
   if (e != cudaSuccess) return bail(e);
   ++kernels;
@@ -596,13 +599,9 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
   ra.E = n_experts;
   ra.k = top_k;
   int g = d->num_sms < hidden / 8 ? d->num_sms : hidden / 8;
-  if (batch > 8) {
-    const int cap = d->num_sms * 8 / batch;
-    g = g < cap ? g : cap;
-  }
   ra.G = g < 1 ? 1 : g;
   const int rows = ceil_div(hidden, ra.G);
-  const int cap_rows = 40960 / (2 * n_experts);
+  const int cap_rows = 65536 / (2 * n_experts + 4 * moe::router_bpad(batch));
   ra.chunk_rows = rows < cap_rows ? rows : cap_rows;
   if (ra.chunk_rows < 1) ra.chunk_rows = 1;
   ra.status = reinterpret_cast<int*>(d->scratch);
@@ -613,12 +612,13 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
   ra.topk_w = topk_w;
   const size_t smem = moe::router_smem_bytes(batch, n_experts, ra.chunk_rows);
   cudaFuncAttributes fa{};
-  if ((e = cudaFuncGetAttributes(&fa, moe::router_topk_kernel)) != cudaSuccess) return fail_cuda(e);
+  const RouterKernel rk = pick_router(n_experts);
+  if ((e = cudaFuncGetAttributes(&fa, rk)) != cudaSuccess) return fail_cuda(e);
   if ((size_t)fa.maxDynamicSharedSizeBytes < smem) {
-    e = cudaFuncSetAttribute(moe::router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail_cuda(e);
   }
-  e = launch(moe::router_topk_kernel, ra.G, moe::kRouterThreads, smem, st, false, ra);
+  e = launch(rk, ra.G, moe::kRouterThreads, smem, st, false, ra);
   if (e != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }
@@ -662,7 +662,7 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
     h->grid_router_max = gr < cap ? gr : cap;
     if (h->grid_router_max < 1) h->grid_router_max = 1;
     const int rows = ceil_div(shapes->hidden, h->grid_router_max);
-    const int cap_rows = 40960 / (2 * shapes->n_experts);
+    const int cap_rows = 65536 / (2 * shapes->n_experts + 4 * moe::router_bpad(shapes->max_batch));
     h->router_chunk_rows = rows < cap_rows ? rows : cap_rows;
     if (h->router_chunk_rows < 1) h->router_chunk_rows = 1;
   }

@@ -41,9 +41,12 @@ struct RouterArgs {
   int* status;
 };
 
+// Tokens padded to a multiple of 8 (x is staged token-contiguous per row).
+__host__ __device__ inline int router_bpad(int B) { return (B + 7) / 8 * 8; }
+
 // Shared memory needed by router_topk_kernel for these sizes.
 __host__ __device__ inline size_t router_smem_bytes(int B, int E, int chunk_rows) {
-  size_t gemv = (size_t)chunk_rows * E * 2 + (size_t)B * chunk_rows * 4;
+  size_t gemv = (size_t)chunk_rows * E * 2 + (size_t)router_bpad(B) * chunk_rows * 4;
   size_t topk = (size_t)kMaxAssign * 8 + (size_t)E * 16 + 64;
   gemv = (gemv + 15) / 16 * 16;
   return gemv > topk ? gemv : topk;
@@ -91,6 +94,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
   return r;
 }
 
+// NV: logits per lane a warp holds in registers during top-k (E <= 32 * NV).
+template <int NV>
 __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __grid_constant__ RouterArgs a) {
   extern __shared__ __align__(1024) uint8_t router_smem[];
   uint8_t* smem = router_smem;
@@ -124,11 +129,14 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
 
   uint32_t phase = 0;
   const int npairs = E / 2;
+  const int bp = router_bpad(B);
   for (int r0 = h0; r0 < h1; r0 += a.chunk_rows) {
     const int nr = min(a.chunk_rows, h1 - r0);
-    for (int i = tid; i < B * nr; i += kRouterThreads) {
-      const int t = i / nr, r = i - t * nr;
-      xs[i] = __bfloat162float(a.x[(size_t)t * H + r0 + r]);
+    // x staged as [row][token] (tokens padded to 8 with zeros), so a row's
+    // 8-token group is two 16-byte shared loads
+    for (int i = tid; i < bp * nr; i += kRouterThreads) {
+      const int r = i / bp, t = i - r * bp;
+      xs[i] = t < B ? __bfloat162float(a.x[(size_t)t * H + r0 + r]) : 0.f;
     }
     mbar_wait_bounded(&bar, phase, a.status);
     phase ^= 1;
@@ -139,16 +147,17 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = 0.f;
         const int nt = min(8, B - t0);
+#pragma unroll 4
         for (int r = 0; r < nr; ++r) {
           float w0, w1;
           bf16x2_to_f32(reinterpret_cast<const uint32_t*>(rs + (size_t)r * E)[p], w0, w1);
+          const float4 xa = *reinterpret_cast<const float4*>(xs + (size_t)r * bp + t0);
+          const float4 xb = *reinterpret_cast<const float4*>(xs + (size_t)r * bp + t0 + 4);
+          const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            if (j < nt) {
-              const float xv = xs[(t0 + j) * nr + r];
-              acc[j][0] = fmaf(xv, w0, acc[j][0]);
-              acc[j][1] = fmaf(xv, w1, acc[j][1]);
-            }
+            acc[j][0] = fmaf(xv[j], w0, acc[j][0]);
+            acc[j][1] = fmaf(xv[j], w1, acc[j][1]);
           }
         }
 #pragma unroll
@@ -184,10 +193,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   const int nv = (E + 31) / 32;
   for (int t = warp; t < B; t += kRouterThreads / 32) {
     float* lg = a.logits + (size_t)t * E;
-    float v[kMaxExperts / 32];
+    float v[NV];
     uint32_t taken = 0;
 #pragma unroll
-    for (int i = 0; i < kMaxExperts / 32; ++i) {
+    for (int i = 0; i < NV; ++i) {
       const int e = lane + 32 * i;
       v[i] = -INFINITY;
       if (i < nv && e < E) {
@@ -195,13 +204,13 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
         __stcg(lg + e, 0.f);
       }
     }
-    int my_id = -1;
-    float my_v = -INFINITY;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+    // each lane keeps its best untaken (value, id); only the lane that owned
+    // a round's winner has to look again
+    auto local_best = [&](float& bv, int& bi) {
+      bv = -INFINITY;
+      bi = 0x7fffffff;
 #pragma unroll
-      for (int i = 0; i < kMaxExperts / 32; ++i) {
+      for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
         // e ascends with i, so strict '>' keeps the smaller id on equal logits
         if (i < nv && e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > bv)) {
@@ -209,15 +218,27 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
           bi = e;
         }
       }
+    };
+    float lbv;
+    int lbi;
+    local_best(lbv, lbi);
+    int my_id = -1;
+    float my_v = -INFINITY;
+    for (int j = 0; j < k; ++j) {
+      float bv = lbv;
+      int bi = lbi;
       warp_argmax(bv, bi);
       if (bi < 0 || bi >= E) {  // cannot happen for k <= E; keep the plan valid
         atomicCAS(a.status, kStatusOk, kStatusPlan);
         bi = j;
       }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
       if (lane == j) {
         my_id = bi;
         my_v = bv;
+      }
+      if ((bi & 31) == lane) {
+        taken |= 1u << (bi >> 5);
+        local_best(lbv, lbi);
       }
     }
     // renormalised weights: p_j / sum_S p = exp(l_j - l_max) / sum_S exp(l_i - l_max)
