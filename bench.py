@@ -4,10 +4,13 @@ HBM GB/s of the distinct weights touched, against the measured B200 peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config full_b1] [--impl reference]
 
-A step is one forward of the whole block (router + top-k + bucketing, routed
-SwiGLU experts, shared expert on the aux stream, combine + residual) over one
-batch of synthetic tokens.  Default workload: the full-size block at batch 1
-(hidden 7168, 384 experts top-8, inter 2048, one shared expert).
+A step is one forward of the whole block (router + top-k + bucketing, shared
+expert, routed SwiGLU experts, combine + residual) over one batch of
+synthetic tokens, in the library's default plan (router kernel, one expert
+kernel for the shared and the routed experts, combine kernel); --two-stream
+times the plan with the shared expert on the aux stream instead.  Default
+workload: the full-size block at batch 1 (hidden 7168, 384 experts top-8,
+inter 2048, one shared expert).
 
 Timing: the forward is captured once in a CUDA graph (both streams) and
 replayed; L2 is flushed (a 2x-L2 write) before every step and each step is
@@ -48,6 +51,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--two-stream", action="store_true",
+                   help="time the plan with the shared expert on the aux stream (MOE_FLAG_TWO_STREAM)")
     return p.parse_args()
 
 
@@ -275,7 +280,7 @@ def run_ours(args):
     wts = synth.make_weights(s, seed=args.seed, device=dev, routing=wl.routing)
     x = synth.make_x(B, s.hidden, seed=args.seed + 1000 * rank).to(dev)
     blk = MoEDecode(s.hidden, s.n_experts, s.top_k, s.inter, s.shared_inter, n_shared=s.n_shared,
-                    max_batch=max(B, 1), router_bias=wts.router_bias)
+                    max_batch=max(B, 1), router_bias=wts.router_bias, two_stream=args.two_stream)
     out = torch.empty_like(x)
     ids = torch.empty(B, s.top_k, dtype=torch.int32, device=dev)
     w = torch.empty(B, s.top_k, dtype=torch.float32, device=dev)
@@ -370,18 +375,28 @@ def run_ours(args):
             if i < 5:
                 continue
             kt["router"].append(evs[0].elapsed_time(evs[1]))
-            kt["experts"].append(evs[1].elapsed_time(evs[2]))
-            kt["combine"].append(evs[2].elapsed_time(evs[3]))
-            kt["shared"].append(evs[4].elapsed_time(evs[5]))
+            if args.two_stream:
+                kt["experts"].append(evs[1].elapsed_time(evs[2]))
+                kt["combine"].append(evs[2].elapsed_time(evs[3]))
+                kt["shared"].append(evs[4].elapsed_time(evs[5]))
+            else:  # one expert kernel: shared + routed experts
+                kt["experts"].append(evs[4].elapsed_time(evs[5]))
+                kt["combine"].append(evs[2].elapsed_time(evs[3]))
             kt["step"].append(evs[0].elapsed_time(evs[3]))
     blk.set_timing_events(None)
-    kern_us = {k: round(1e3 * statistics.mean(v), 2) for k, v in kt.items()}
+    kern_us = {k: round(1e3 * statistics.mean(v), 2) for k, v in kt.items() if v}
     peak, peak_kind = peaks()
-    # dominant kernel: the routed experts (UP + SwiGLU + DOWN of every active expert)
-    exp_bytes = distinct * s.expert_bytes()
+    # dominant kernel: the expert kernel.  Default plan: shared expert + every
+    # active routed expert (UP + SwiGLU + DOWN); two-stream plan: the routed
+    # experts only.
+    exp_bytes = distinct * s.expert_bytes() + (0 if args.two_stream else s.shared_bytes())
     exp_gbs = exp_bytes / (kern_us["experts"] * 1e-6) / 1e9
-    traffic = ncu_traffic("expert_mlp_routed", wl.name)
-    roofline = {"bound": "hbm", "kernel": "expert_mlp_kernel<routed>", "achieved": round(exp_gbs, 1),
+    kname = "expert_mlp_routed" if args.two_stream else "expert_mlp"
+    traffic = ncu_traffic(kname, wl.name)
+    roofline = {"bound": "hbm",
+                "kernel": "expert_mlp_kernel<routed only>" if args.two_stream
+                else "expert_mlp_kernel<shared + routed>",
+                "achieved": round(exp_gbs, 1),
                 "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(exp_gbs / peak, 4),
                 "traffic": traffic, "algorithmic_bytes_per_launch": exp_bytes,
                 "launch_us": kern_us["experts"],
@@ -432,7 +447,7 @@ def run_ours(args):
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": _config_dict(wl),
+            "config": dict(_config_dict(wl), plan="two_stream" if args.two_stream else "default"),
             "us_per_block": round(ms_per_step * 1e3, 2), "tokens_per_s": round(B * 1e3 / ms_per_step, 1),
             "bytes_per_step": bstep, "distinct_experts": distinct,
             "roofline": roofline, "kernels_us": kern_us, "cpu_baseline": cpu, "e2e": e2e,

@@ -11,8 +11,19 @@
  *   3. per selected expert, the SwiGLU up projection
  *      a = silu(x . W13[:, :I]) * (x . W13[:, I:]);
  *   4. the down projection y = a . W2, weighted by the routing weight;
- *   5. the shared expert (same MLP, weight 1) on the auxiliary stream;
+ *   5. the shared expert (same MLP, weight 1), overlapping steps 1-2;
  *   6. out = x + sum_j w_j y_j + shared, rounded once to bf16.
+ *
+ * Two execution plans (chosen per handle by moe_decode_shapes.flags):
+ *   default: three kernels on stream_main.  The router kernel (steps 1-2);
+ *     one persistent expert kernel that streams the shared expert's up
+ *     projection first -- it needs nothing from the router, so it runs while
+ *     the router is still working (programmatic dependent launch) -- then the
+ *     routed experts and the shared expert's down projection; the combine
+ *     (step 6).  stream_aux is not used.
+ *   MOE_FLAG_TWO_STREAM: the pages' layout.  Router and routed experts on
+ *     stream_main, the shared expert on stream_aux (forked and joined with
+ *     events), then a separate combine kernel.
  *
  * The steps follow the pages "Hyper Optimizing Kimi K3 in vLLM: Moving Fast
  * and Responsibly" (commentary; section "Recovering time between operators":
@@ -70,8 +81,10 @@ extern "C" {
  * router_bias (optional) is a device float32 [n_experts] added to the router
  * logits before softmax and selection; NULL means no bias.  It is read by
  * every forward (the pointer is kept, the data is not copied).
- * flags is reserved and must be 0.
+ * flags: 0 or MOE_FLAG_TWO_STREAM (see the top of this file); other bits
+ * are rejected with MOE_ERR_UNSUPPORTED_SHAPE.
  */
+#define MOE_FLAG_TWO_STREAM 1u
 typedef struct moe_decode_shapes {
   int32_t hidden;
   int32_t n_experts;
@@ -90,8 +103,9 @@ typedef struct moe_decode_ctx* moe_decode_t;
  * Per-handle counters (host side), filled by moe_decode_get_stats.
  *   forwards          : successful forwards enqueued by this handle
  *   kernels_launched  : kernels enqueued by this handle since creation
- *   last_kernels      : kernels enqueued by the last forward (4, or 3 without
- *                       a shared expert)
+ *   last_kernels      : kernels enqueued by the last forward (default plan:
+ *                       3; MOE_FLAG_TWO_STREAM: 4, or 3 without a shared
+ *                       expert)
  *   last_token_tiles  : token tiles of 8 the expert kernels were prepared for
  *                       in the last forward (ceil(batch / 8))
  */
@@ -116,9 +130,11 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle);
  * Enqueue one forward of the block on stream_main / stream_aux (cudaStream_t
  * passed as void*; NULL is the legacy default stream).  Asynchronous, does no
  * host synchronisation and allocates nothing, so it can be captured in a
- * CUDA graph.  The shared expert is forked onto stream_aux with an event and
- * joined back; when the call returns every piece of work is ordered before
- * anything later enqueued on stream_main.  stream_aux may equal stream_main.
+ * CUDA graph.  With MOE_FLAG_TWO_STREAM the shared expert is forked onto
+ * stream_aux with an event and joined back (stream_aux may equal
+ * stream_main); by default stream_aux is ignored (it may be NULL).  When the
+ * call returns every piece of work is ordered before anything later enqueued
+ * on stream_main.
  *
  *   x          device bf16 [batch, hidden]          block input and residual
  *   router_w   device bf16 [hidden, n_experts]      router weights (in x out)
@@ -184,12 +200,15 @@ const char* moe_decode_last_cuda_error_string(void);
 /*
  * Per-kernel timing.  events: HOST array of MOE_TIMING_EVENTS cudaEvent_t
  * (passed as void*) created by the caller with timing enabled, or NULL to
- * switch timing off.  While set, every forward records, on stream_main,
+ * switch timing off.  While set, every forward records, with
+ * MOE_FLAG_TWO_STREAM, on stream_main
  *   [0] before the router, [1] after the router, [2] after the routed
  *   experts (up + SwiGLU + down), [3] after the combine,
  * and on stream_aux
- *   [4] before the shared expert, [5] after it,
- * so cudaEventElapsedTime gives each kernel's duration.  Recording an event
+ *   [4] before the shared expert, [5] after it;
+ * with the default plan (all on stream_main) [0] before the router, [1] and
+ * [4] after it, [2] and [5] after the expert kernel (shared + routed
+ * experts), [3] after the combine.  cudaEventElapsedTime gives each kernel's duration.  Recording an event
  * between two kernels also makes the second wait for the first to finish
  * (no early launch), so timed forwards can be slightly slower.  The handle
  * keeps the array's values (not the pointer); the caller keeps the events

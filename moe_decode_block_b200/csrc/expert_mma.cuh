@@ -1,82 +1,97 @@
-// expert_mma.cuh -- grouped expert SwiGLU MLPs (up + SwiGLU + down) streamed
-// from HBM with TMA, multiplied on the tensor cores, in one persistent launch.
+// expert_mma.cuh -- the expert SwiGLU MLPs of the block (shared expert and
+// routed experts: up + SwiGLU + down) streamed from HBM with TMA, multiplied
+// on the tensor cores, in one persistent launch.
 //
 // Pages: "Hyper Optimizing Kimi K3 in vLLM: Moving Fast and Responsibly"
 // (commentary), section "Recovering time between operators": small-batch
 // decode waits on weight reads; small-matrix projection kernels at batch 1-2
-// and split-K at larger batches expose enough parallel work; weights are
-// loaded before their consumer starts, and dependent work should begin as
-// soon as its inputs exist.  The pages' kernels were written for GB300 in
-// CuTe DSL; this is a B200 design of the same ideas.
+// and split-K at larger batches expose enough parallel work; the shared
+// expert overlaps routing; weights are loaded before their consumer starts;
+// dependent work should begin as soon as its inputs exist; the residual add
+// belongs in the producing step's epilogue.  The pages' kernels were written
+// for GB300 in CuTe DSL; this is a B200 design of the same ideas.
 //
-// What one launch computes (routed: every active expert of the plan; DENSE:
-// the shared expert over all tokens, weight 1):
-//   UP   h[slot, :] = x[tok, :] . W13[e]           (fp32, split-K partial sums)
-//        a[slot, c] = bf16(silu(h[slot, c]) * h[slot, I + c])  per panel, once complete
-//   DOWN acc[tok, :] += w_slot * a[slot, :] . W2[e] (fp32 atomics)
+// What one launch computes, per unit (one expert's weights over at most 32
+// tokens):
+//   UP   h[row, :] = x[tok, :] . W13           (fp32, split-K partial sums)
+//        a[row, c] = bf16(silu(h[row, c]) * h[row, I + c])  per panel, once complete
+//   DOWN acc[tok, :] += w * a[row, :] . W2      (fp32 atomics)
+// Shared-expert units take the tokens 32u .. 32u + 31 with weight 1 (rows of
+// h_s / a_s are token indices); routed units come from the router's plan
+// (rows of h / a are assignment slots b * k + j, weight = routing weight).
+//
+// Work list, in two segments:
+//   A: UP stages of the shared expert's units;
+//   B: UP stages of the routed units, DOWN stages of the shared units, DOWN
+//      stages of the routed units.
+// Segment A needs nothing from the router, so it runs *before* the
+// grid-dependency wait and overlaps the router kernel (launched just before
+// this one under programmatic dependent launch); a producer calls the wait
+// only when its ticket reaches segment B, whose length it then reads from the
+// plan.  CTAs pull chunks of stages from a global ticket counter.  Segment A
+// goes out in one round of a chunk per CTA; in segment B the first three
+// quarters go out in chunks of T/(4G) stages (at most 64),
+// the next 3/16 in quarter chunks, the rest one at a time, so the grid needs
+// no co-residency and ends with a tail of about one stage.  A DOWN stage
+// reads activation rows [row0, row0 + R), which one UP panel of its unit
+// produces; it is issued once that panel is published (a per-panel flag
+// holding the launch epoch, so flags never need clearing).  Every UP stage is
+// handed out before any DOWN stage, so the CTAs that still owe UP work are
+// running and the wait always ends (it is bounded all the same).  The shared
+// expert's DOWN stages would wait for its UP panels if they followed them in
+// segment A (a CTA that starts late, on the SM where the router's last CTA
+// ran, can hold the last of them); after the routed UP stages they are ready.
+// The producer keeps the plan (unit list, assignment slots) and the panels it
+// has seen published in shared memory: at every chunk change it would
+// otherwise walk the plan with chains of dependent L2 reads, and as all CTAs
+// change chunks at about the same time, those stalls line up into dips of
+// the whole GPU's bandwidth.
 //
 // Panels.  Each matrix is cut into column panels and K-row stages.  A
 // consumer thread keeps at most 128 fp32 accumulators, so panel columns x
-// token tiles is bounded: a unit (expert) with n tokens uses the widest panel
-// its token count allows --
-//   class 0: n <=  8 : 2048 local columns, 16-row stages (1 token tile, 64 accumulators)
+// token tiles is bounded; a unit with n tokens uses the widest panel its
+// token count allows --
+//   class 0: n <=  8 : 2048 local columns, 16-row stages (1 token tile)
 //   class 1: n <= 16 : 2048 local columns, 16-row stages (2 token tiles)
 //   class 2: n <= 32 : 1024 local columns, 32-row stages (4 token tiles)
-//   class 3: n <= 64 :  512 local columns, 64-row stages (8 token tiles)
 // -- every stage is 64 KB of weights.  A launch is compiled for the largest
 // class its batch can produce (KC), so batches of <= 8 tokens run code that
-// holds only 64 accumulators.  Wide panels matter because the TMA
-// engine pays per copy: a stage is one bulk copy per panel row (two for UP,
-// whose panels pair gate columns [c0, c0+LW/2) with up columns [I+c0, ...),
-// so a panel holds both halves of its SwiGLU), and rows of 2-4 KB stream at
-// full HBM rate where 0.5-1 KB rows do not.
-//
-// Work list.  [UP stages of every unit, then DOWN stages of every unit]; CTAs
-// pull chunks from a global ticket counter.  Ticket i maps to a fixed range:
-// the first three quarters of the list go out in chunks of T/(4G) stages (at
-// most 64), the rest one stage at a time, so the grid needs no co-residency
-// and ends with a tail of about one stage.  A DOWN stage reads rows
-// [row0, row0 + R) of the unit's activations, which one UP panel produces;
-// it is issued once that panel is published (a per-panel flag holding the
-// launch epoch, so flags never need clearing).  Every UP stage was handed out
-// before any DOWN stage, so the CTAs that still owe UP work are running and
-// the wait always ends (it is bounded all the same).
+// holds only 32 accumulators per thread (with 16 consumer warps).  UP panels
+// pair gate columns [c0, c0 + LW/2) with up columns [I + c0, ...), so a panel
+// holds both halves of its SwiGLU.
 //
 // Data movement.  One producer warp fills a shared-memory ring of 64 KB
 // stages, guarded by mbarriers, with TMA (no multicast, L2 evict-first):
 //  * tensor-map path (hidden and intermediate sizes multiples of 64): each
-//    expert matrix has a tensor map over the 3-D view {64 columns, rows,
-//    column chunks of 64}; one tiled load moves a {64, 16, 4} box (16 rows x
-//    256 columns, 8 KB) with 128-byte swizzling, so a stage takes 8 loads and
-//    the swizzle makes the ldmatrix reads conflict-free.  The TMA engine pays
-//    a fixed cost per operation, so few large loads keep it ahead of HBM.
+//    matrix has a tensor map over the 3-D view {64 columns, rows, column
+//    chunks of 64}; one tiled load moves a {64, 16, 4} box (16 rows x 256
+//    columns, 8 KB) with 128-byte swizzling, so a stage takes 8 loads and the
+//    swizzle makes the ldmatrix reads conflict-free.  The TMA engine pays a
+//    fixed cost per operation, so few large loads keep it ahead of HBM.
 //  * row-copy path (other shapes): one cp.async.bulk per panel row (two for
 //    UP), into rows padded by 16 bytes for the same reason.
 // Plus one small copy per token of the stage's activations (x for UP, bf16 a
-// for DOWN), all counted on the stage's mbarrier, and a stage header.  Eight consumer warps split
-// the panel's columns and run mma.sync.m16n8k16 (bf16 in, fp32 accumulate)
-// with the tokens as the N dimension, so the tensor cores do the arithmetic
-// and the consumers stay far ahead of HBM.  Partial sums of a piece
-// (consecutive stages of one panel) are flushed with fp32 atomics; for UP the
-// last warp to contribute to a panel (per-panel counter of warp-stages)
-// applies the SwiGLU, returns its accumulators to zero and publishes the
-// panel to DOWN.  The consumer loop has no CTA-wide barrier, so a warp whose
-// bounded wait gives up can never leave another warp blocked.
-//
-// Ordering under programmatic dependent launch: the plan, activations and
-// workspace are read only after the grid-dependency wait.
+// for DOWN), all counted on the stage's mbarrier, and a stage header.  The
+// consumer warps split the panel's columns and run mma.sync.m16n8k16 (bf16
+// in, fp32 accumulate) with the tokens as the N dimension.  Partial sums of a
+// piece (consecutive stages of one panel) are flushed with fp32 atomics; for
+// UP the last warp to contribute to a panel (per-panel counter of
+// warp-stages) applies the SwiGLU, returns its accumulators to zero and
+// publishes the panel to DOWN.  The consumer loop has no CTA-wide barrier, so
+// a warp whose bounded wait gives up can never leave another warp blocked.
 #pragma once
 
 #include "moe_device.cuh"
 
 namespace moe {
 
-constexpr int kMaxTok = 64;
-constexpr int kNumClasses = 4;
-__host__ __device__ constexpr int class_lw(int c) { return c <= 1 ? 2048 : (c == 2 ? 1024 : 512); }
-__host__ __device__ constexpr int class_rows(int c) { return c <= 1 ? 16 : (c == 2 ? 32 : 64); }
-__host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : (c == 2 ? 4 : 8)); }
-__host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : (n <= 32 ? 2 : 3)); }
+constexpr int kUnitTok = kMaxUnitTokens;  // tokens of one unit, at most
+constexpr int kNumClasses = 3;
+__host__ __device__ constexpr int class_lw(int c) { return c <= 1 ? 2048 : 1024; }
+__host__ __device__ constexpr int class_rows(int c) { return c <= 1 ? 16 : 32; }
+__host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : 4); }
+// class of a unit with n <= kUnitTok tokens
+__host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : 2); }
 // Consumer warps of the instance compiled for classes <= kc: sixteen when a
 // thread needs only 32 accumulators (more warps hide more latency), eight
 // otherwise -- nine warps per CTA leave each thread 168 registers, enough for
@@ -90,69 +105,145 @@ __host__ __device__ constexpr int acc_frags(int kc) {
   return kc == 0 ? class_mt(0, consumer_warps_for(0)) * class_nt(0)
                  : class_mt(1, consumer_warps_for(kc)) * class_nt(1);
 }
-constexpr int kStageWBytes = 65536 + 64 * 16;              // rows * (2*LW + 16), largest over classes
-constexpr int kStageXBytes = kMaxTok * (64 * 2 + 16);      // tokens * (2*rows + 16), largest
-constexpr int kStageBytesMma = kStageWBytes + kStageXBytes;  // 75776
+static_assert(class_mt(2, 8) * class_nt(2) == acc_frags(2), "class 2 fits the class 1 budget");
+constexpr int kStageWBytes = 65536 + 32 * 16;                // rows * (2*LW + 16), largest over classes
+constexpr int kStageXBytes = kUnitTok * (32 * 2 + 16);       // tokens * (2*rows + 16), largest
+constexpr int kStageBytesMma = kStageWBytes + kStageXBytes;  // 68608 = 67 KB (stages stay 1 KB aligned)
+static_assert(kStageBytesMma % 1024 == 0, "128-byte swizzle atoms need 1 KB aligned stages");
 constexpr int kMaxStagesMma = 3;
 constexpr int kMaxChunk = 64;  // stages per queue grab, at most
 // tensor-map path: boxes of {64 columns, 16 rows, 4 column chunks}
 constexpr int kChunkCols = 64;
 constexpr int kBoxRows = 16;
 constexpr int kBoxChunks = 4;
-constexpr int kChunkTile = kBoxRows * kChunkCols * 2;          // 2048 B: one chunk of one 16-row block
-constexpr int kBoxBytes = kChunkTile * kBoxChunks;               // 8192 B per load
+constexpr int kChunkTile = kBoxRows * kChunkCols * 2;  // 2048 B: one chunk of one 16-row block
+constexpr int kBoxBytes = kChunkTile * kBoxChunks;     // 8192 B per load
 constexpr int kTensorMapBytes = 128;
-// UP panels of a unit, at most: ceil(I / 256) (class 3); sizes the panel counters
-__host__ __device__ inline int max_up_panels(int I) { return (I + class_lw(3) / 2 - 1) / (class_lw(3) / 2); }
+// UP panels of a unit, at most: ceil(I / 512) (class 2); sizes the panel counters
+__host__ __device__ inline int max_up_panels(int I) { return (I + class_lw(2) / 2 - 1) / (class_lw(2) / 2); }
 
 enum : int { kKindUp = 0, kKindDown = 1, kKindEnd = 2 };
 enum : int { kFirst = 1, kLast = 2 };
 
 // Stage header, written by the producer before it arms the stage's barrier.
-// row[n]: UP -> the h/a row (assignment slot) of token n of the unit;
-//         DOWN -> the output row (token).  wt[n]: DOWN routing weight.
+// row[n]: UP -> the h row of token n of the unit; DOWN -> the output row
+// (token).  wt[n]: DOWN weight.  seg: 0 shared expert, 1 routed.
 struct StageHdr {
-  int kind, unit, cls, cp, row0, nrows, flags, ntok, begin, pstages;  // pstages: stages of the piece (on its last)
-  int row[kMaxTok];
-  float wt[kMaxTok];
+  int kind, seg, unit, cls, cp, row0, nrows, flags, ntok, pstages, pad_[2];  // pstages: stages of the piece (on its last)
+  int row[kUnitTok];
+  float wt[kUnitTok];
 };
 
 struct MmaArgs {
   int H;             // hidden (UP rows, DOWN columns)
-  int I;             // intermediate (UP columns per half, DOWN rows)
+  int I;             // routed intermediate
+  int Is;            // shared intermediate
+  int E;             // routed experts (bounds the plan's expert ids)
+  int top_k;         // bounds the plan's assignment slots
   int n_stages;      // ring depth
-  int batch;         // tokens (DENSE)
+  int batch;         // tokens
+  int n_su;          // shared-expert units: ceil(batch / 32), or 0 for no shared expert
+  int has_routed;    // 1: routed units too (their plan comes from the previous grid)
   int max_units;     // bound on the plan's n_active
-  int panel_stride;  // panel counters per unit (max_up_panels(I))
-  const __nv_bfloat16* w13;  // DENSE weights; routed experts come from the pointer tables
-  const __nv_bfloat16* w2;
-  const uint8_t* maps13;     // tensor-map path: [units] 128-byte maps of w13 (DENSE: one)
-  const uint8_t* maps2;      // tensor-map path: maps of w2
-  const Plan* plan;          // nullptr for DENSE
+  int panel_stride;  // routed panel counters per unit (max_up_panels(I))
+  int panel_stride_s;
+  const __nv_bfloat16* w13_s;  // shared expert weights (routed ones come from the pointer tables)
+  const __nv_bfloat16* w2_s;
+  const uint8_t* maps13;     // tensor-map path: [E] 128-byte maps of the routed w13
+  const uint8_t* maps2;      // [E] maps of the routed w2
+  const uint8_t* maps13_s;   // shared expert maps
+  const uint8_t* maps2_s;
+  const Plan* plan;
   const __nv_bfloat16* x;    // [B, H]
-  float* h;                  // [slots, 2I] fp32, zero between calls
-  __nv_bfloat16* a;          // [slots, I] bf16
-  float* acc;                // [B, H] fp32 output accumulator
+  float* h;                  // [B*k, 2I] fp32, zero between calls
+  __nv_bfloat16* a;          // [B*k, I] bf16
+  float* h_s;                // [B, 2Is]
+  __nv_bfloat16* a_s;        // [B, Is]
+  float* acc;                // [B, H] fp32 output accumulator, zero between calls
   unsigned* panel_cnt;       // [units * panel_stride] finished warp-stages per UP panel, zero between calls
   unsigned* panel_ready;     // [units * panel_stride] = epoch + 1 once the UP panel's activations are written
+  unsigned* panel_cnt_s;     // shared expert: [n_su * panel_stride_s]
+  unsigned* panel_ready_s;
   unsigned* queue;           // [0] ticket counter, [1] finished CTAs (zero between calls), [2] launch epoch
   int* status;
 };
 
+// Producer's copy of the plan in shared memory: per unit the expert id,
+// first assignment and token count; per assignment its slot (b * k + j, from
+// which the token is b = slot / k); per unit (routed, then shared) the bit
+// mask of its UP panels seen published.
+constexpr int kMaxSharedUnits = kMaxBatch / kUnitTok;
+constexpr int kPlanCacheBytes =
+    (kMaxUnits * (2 + 2 + 1) + kMaxAssign * 2 + 3) / 4 * 4 + (kMaxUnits + kMaxSharedUnits) * 4;
+
 __host__ __device__ inline size_t mma_smem_bytes(int n_stages) {
   // + 1 KB so the ring can start on a 1024-byte boundary (128-byte swizzle)
   return 1024 + (size_t)n_stages * kStageBytesMma + 2 * kMaxStagesMma * sizeof(uint64_t) +
-         kMaxStagesMma * sizeof(StageHdr) + 16 * sizeof(int);
+         kMaxStagesMma * sizeof(StageHdr) + 16 * sizeof(int) + kPlanCacheBytes;
 }
 
-// Panels and stages per panel of one unit with class `cls`, UP or DOWN list.
-__device__ __forceinline__ int unit_panels(int cls, bool up, int H, int I) {
+// Panels and stages per panel of one unit with class `cls`, UP or DOWN list
+// (I: the unit's intermediate size).
+__host__ __device__ __forceinline__ int unit_panels(int cls, bool up, int H, int I) {
   const int lw = class_lw(cls);
   return up ? (I + lw / 2 - 1) / (lw / 2) : (H + lw - 1) / lw;
 }
-__device__ __forceinline__ int unit_panel_stages(int cls, bool up, int H, int I) {
+__host__ __device__ __forceinline__ int unit_panel_stages(int cls, bool up, int H, int I) {
   const int r = class_rows(cls);
   return up ? (H + r - 1) / r : (I + r - 1) / r;
+}
+__host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int I) {
+  return unit_panels(cls, up, H, I) * unit_panel_stages(cls, up, H, I);
+}
+
+// Ticket schedule over a segment of T stages for a grid of G CTAs: 3/4 of
+// the list in chunks of c_big = T / (div * G), then 3/16 in chunks of
+// c_big / 4, then single stages (make_sched); or one round of at most G
+// chunks of max(1, T / G) stages plus the remainder (make_round).
+struct Sched {
+  int T, c_big, c_mid, n_big, n_mid, T1, T2, n_tickets;
+};
+__device__ __forceinline__ Sched make_round(int T, int G) {
+  Sched s;
+  s.T = T;
+  const int c = T / G > 1 ? T / G : 1;  // every CTA gets a chunk before any gets a second
+  s.c_big = c;
+  s.n_big = T / c;
+  s.T1 = s.n_big * c;
+  s.c_mid = T - s.T1 > 0 ? T - s.T1 : 1;  // the remainder, as one more chunk
+  s.n_mid = T - s.T1 > 0 ? 1 : 0;
+  s.T2 = T;
+  s.n_tickets = s.n_big + s.n_mid;
+  return s;
+}
+__device__ __forceinline__ Sched make_sched(int T, int G, int div) {
+  Sched s;
+  s.T = T;
+  int c = T / (div * G);
+  c = c < 1 ? 1 : (c > kMaxChunk ? kMaxChunk : c);
+  s.c_big = c;
+  s.c_mid = c / 4 < 1 ? 1 : c / 4;
+  s.n_big = (T / 4 * 3) / c;
+  s.T1 = s.n_big * c;
+  s.n_mid = ((T - s.T1) / 4 * 3) / s.c_mid;
+  s.T2 = s.T1 + s.n_mid * s.c_mid;
+  s.n_tickets = s.n_big + s.n_mid + (T - s.T2);
+  return s;
+}
+// stages [b, e) of ticket tk (0 <= tk < n_tickets)
+__device__ __forceinline__ void sched_range(const Sched& s, int tk, int& b, int& e) {
+  if (tk < s.n_big) {
+    b = tk * s.c_big;
+    e = b + s.c_big;
+  } else if (tk - s.n_big < s.n_mid) {
+    b = s.T1 + (tk - s.n_big) * s.c_mid;
+    e = b + s.c_mid;
+  } else {
+    b = s.T2 + (tk - s.n_big - s.n_mid);
+    e = b + 1;
+  }
+  if (b > s.T) b = s.T;
+  if (e > s.T) e = s.T;
 }
 
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -199,7 +290,7 @@ __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint
     if (k0 >= nrows) break;
     const bool half = (nrows - k0) < 16;  // only 8 valid rows in this k-step
     // token fragments: kept for all tiles when there are few of them, loaded
-    // per m-tile otherwise (keeps the 64 accumulators in registers)
+    // per m-tile otherwise (keeps the accumulators in registers)
     constexpr bool kKeepB = NT <= 2;
     uint32_t b[kKeepB ? NT : 1][2];
     auto load_b = [&](int nt, uint32_t& b0, uint32_t& b1) {
@@ -247,10 +338,9 @@ __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint
   }
 }
 
-// Flush this warp's partial sums of a piece (class C) with fp32 atomics.
-// Local columns: DOWN [0, w) -> c0 + l; UP gate [0, w) -> c0 + l and up
-// [uoff, uoff + w) -> I + c0 + (l - uoff); anything else is padding.  w and
-// uoff are multiples of 8, so four consecutive local columns map to four
+// Local columns of a stage: DOWN [0, w) -> c0 + l; UP gate [0, w) -> c0 + l
+// and up [uoff, uoff + w) -> I + c0 + (l - uoff); anything else is padding.
+// w and uoff are multiples of 8, so four consecutive local columns map to four
 // consecutive output columns.
 __device__ __forceinline__ int local_to_col(int l, bool up, int c0, int w, int uoff, int I) {
   if (!up) return l < w ? c0 + l : -1;
@@ -259,32 +349,36 @@ __device__ __forceinline__ int local_to_col(int l, bool up, int c0, int w, int u
   return -1;
 }
 
-// Flush this warp's partial sums of a piece (class C) with fp32 atomics.  An
-// m-tile's C fragment spreads 16 columns of a token over 8 lanes; shuffles
-// gather each run of 4 columns into one lane, so every 16 bytes take one
-// vector atomic instead of four scalar ones.
+// Flush this warp's partial sums of a piece (class C) with fp32 atomics into
+// rows base + row(n) * ld, where lane n of the warp holds row(n) in my_row and
+// the weight in my_wt (copied from the stage header, so the stage's slot can
+// be handed back before the flush).  An m-tile's C fragment spreads 16
+// columns of a token over 8 lanes; shuffles gather each run of 4 columns into
+// one lane, so every 16 bytes take one vector atomic instead of four scalar
+// ones.
 template <int C, int NF, int CW>
-__device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], const MmaArgs& args, const StageHdr& hd,
-                                            bool up, int c0, int w, int uoff, int LW, int warp, int lane) {
+__device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], float* base, size_t ld, int my_row,
+                                            float my_wt, int ntok, bool up, int c0, int w, int uoff, int LW, int I,
+                                            int warp, int lane) {
   constexpr int MT = class_mt(C, CW), NT = class_nt(C);
   const int m0 = warp * MT * 16;
   if (m0 >= LW) return;
   const int gid = lane >> 2, tig = lane & 3;
-  const int I = args.I, H = args.H;
-  const int ntiles = (hd.ntok + 7) >> 3;
+  const int ntiles = (ntok + 7) >> 3;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     if (nt >= ntiles) break;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int n = nt * 8 + tig * 2 + e;  // this lane's token (same for its tig group)
-      const bool valid = n < hd.ntok;
+      const bool valid = n < ntok;
+      const int r = __shfl_sync(0xffffffffu, my_row, n);
+      const float wr = __shfl_sync(0xffffffffu, my_wt, n);
       float* row = nullptr;
       float wt = 1.f;
       if (valid) {
-        const int r = hd.row[n];
-        wt = up ? 1.f : hd.wt[n];
-        row = up ? args.h + (size_t)r * (2 * I) : args.acc + (size_t)r * H;
+        row = base + (size_t)r * ld;
+        wt = up ? 1.f : wr;
       }
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
@@ -311,7 +405,7 @@ __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], const Mma
   }
 }
 
-template <bool DENSE, int KC, bool TMAP>
+template <int KC, bool TMAP>
 __global__ void __launch_bounds__(expert_threads(KC), 1)
     expert_mlp_kernel(const __grid_constant__ MmaArgs args, const __grid_constant__ ExpertTable tab13,
                       const __grid_constant__ ExpertTable tab2) {
@@ -324,6 +418,12 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   StageHdr* hdr = reinterpret_cast<StageHdr*>(empty + kMaxStagesMma);
   volatile int* s_misc = reinterpret_cast<volatile int*>(hdr + kMaxStagesMma);
   // s_misc[0]: abort flag (a bounded wait gave up), [2]: stages issued
+  uint16_t* s_uexp = reinterpret_cast<uint16_t*>(const_cast<int*>(s_misc) + 16);  // [kMaxUnits]
+  uint16_t* s_ubeg = s_uexp + kMaxUnits;                                          // [kMaxUnits]
+  uint16_t* s_aslot = s_ubeg + kMaxUnits;                                         // [kMaxAssign]
+  uint8_t* s_ucnt = reinterpret_cast<uint8_t*>(s_aslot + kMaxAssign);             // [kMaxUnits]
+  uint32_t* s_ready = reinterpret_cast<uint32_t*>(                                // [kMaxUnits + shared]
+      reinterpret_cast<uint8_t*>(s_uexp) + (kMaxUnits * (2 + 2 + 1) + kMaxAssign * 2 + 3) / 4 * 4);
 
   constexpr int CW = consumer_warps_for(KC);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -340,149 +440,182 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   }
   __syncthreads();
 
-  const int H = args.H, I = args.I;
+  const int H = args.H;
   volatile int* abort_flag = s_misc;
-  const Plan* plan = args.plan;
-  // Launch epoch: advanced by the last CTA of the previous launch (an earlier
-  // grid on this stream), so every CTA of this launch reads the same value.
+  // Launch epoch: advanced by the last CTA of the previous launch on this
+  // workspace, which finished before the previous grid (the router) passed
+  // its own dependency wait; every CTA of this launch reads the same value.
+  const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
 
   if (is_producer) {
     // ================================================================ producer
     const uint64_t pol = l2_evict_first_policy();
-    // The first ticket only touches this kernel's own counter (returned to
-    // zero by the previous launch of this kernel, which finished before the
-    // router started), so take it before the wait: its round trip overlaps
-    // the router's tail.  It is turned into a range only after the wait.
+    const int G = gridDim.x;
+    const int B = args.batch;
+    // The ticket counter was returned to zero by the previous launch (see
+    // the epoch above), so the first ticket is taken at once.
     int tk = 0;
     if (lane == 0) tk = (int)atomicAdd(&args.queue[0], 1u);
-    cudaGridDependencySynchronize();  // the plan and the activations come from earlier kernels
-    const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
-    int n_units = 1;
-    if (!DENSE) {
-      n_units = plan->n_active;
-      if (n_units < 0 || n_units > args.max_units) {
-        if (lane == 0) atomicCAS(args.status, kStatusOk, kStatusPlan);
-        n_units = 0;
-      }
-    }
-    auto unit_tokens = [&](int u) {
-      const int n = DENSE ? args.batch : plan->unit_count[u];
-      return n > kMaxTok ? kMaxTok : n;  // cannot exceed: batch <= 64
-    };
-    auto unit_class = [&](int n) {
+    auto cls_of = [&](int n) {
       const int c = class_for_tokens(n);
-      return c > KC ? KC : c;  // cannot exceed: KC is the class of the batch size
+      return c > KC ? KC : c;  // cannot exceed: KC is the class of min(batch, 32)
     };
-    auto unit_stages = [&](int u, bool up) {
-      const int c = unit_class(unit_tokens(u));
-      return unit_panels(c, up, H, I) * unit_panel_stages(c, up, H, I);
-    };
-    int T_up = 0, T_dn = 0;  // at most ~1.5M stages: 32-bit arithmetic
-    for (int u = lane; u < n_units; u += 32) {
-      T_up += unit_stages(u, true);
-      T_dn += unit_stages(u, false);
+    auto su_tokens = [&](int su) { return min(kUnitTok, B - su * kUnitTok); };
+    auto plan_tokens = [&](int u) { return (int)s_ucnt[u]; };  // valid once segment B is known
+    for (int i = lane; i < kMaxUnits + kMaxSharedUnits; i += 32) s_ready[i] = 0u;
+    __syncwarp();
+    // the shared expert's stages are known without the router
+    int S_up = 0, S_dn = 0;
+    for (int su = 0; su < args.n_su; ++su) {
+      const int c = cls_of(su_tokens(su));
+      S_up += unit_stages(c, true, H, args.Is);
+      S_dn += unit_stages(c, false, H, args.Is);
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      T_up += __shfl_xor_sync(0xffffffffu, T_up, off);
-      T_dn += __shfl_xor_sync(0xffffffffu, T_dn, off);
-    }
-    const int T_all = T_up + T_dn;
-    const int G = gridDim.x;
-    // ticket -> range: 3/4 of the list in chunks of c_big, then 3/16 in
-    // chunks of c_big / 4, then single stages
-    int c_big = T_all / (4 * G);
-    c_big = c_big < 1 ? 1 : (c_big > kMaxChunk ? kMaxChunk : c_big);
-    const int c_mid = c_big / 4 < 1 ? 1 : c_big / 4;
-    const int n_big = (T_all / 4 * 3) / c_big;
-    const int T1 = n_big * c_big;
-    const int n_mid = ((T_all - T1) / 4 * 3) / c_mid;
-    const int T2 = T1 + n_mid * c_mid;
-    auto chunk_of = [&](int tk, int& b, int& e) {
-      if (tk < n_big) {
-        b = tk * c_big;
-        e = b + c_big;
-      } else if (tk - n_big < n_mid) {
-        b = T1 + (tk - n_big) * c_mid;
-        e = b + c_mid;
-      } else {
-        b = T2 + (tk - n_big - n_mid);
-        e = b + 1;
+    const int S_A = S_up;  // segment A: the shared UP stages
+    const Sched sch_A = make_round(S_up, G);
+    // segment B: the routed units, read from the plan once a ticket reaches it
+    Sched sch_B = make_sched(S_dn, G, 4);
+    bool b_known = !args.has_routed;
+    int n_units_r = 0;
+    auto know_b = [&]() {
+      cudaGridDependencySynchronize();  // the plan is written by the router kernel
+      const Plan* pl = args.plan;
+      int n = __ldcg(&pl->n_active);
+      if (n < 0 || n > args.max_units) {
+        if (lane == 0) atomicCAS(args.status, kStatusOk, kStatusPlan);
+        n = 0;
       }
-      if (b > T_all) b = T_all;
-      if (e > T_all) e = T_all;
+      n_units_r = n;
+      // copy the plan to shared memory, sanitised: an entry the router never
+      // produces is flagged and replaced by one that keeps every access in
+      // bounds
+      const int nas = B * args.top_k;
+      bool bad = false;
+      int T = 0;  // at most ~0.5M stages: 32-bit arithmetic
+      for (int u = lane; u < n; u += 32) {
+        int cnt = __ldcg(&pl->unit_count[u]);
+        int ex = __ldcg(&pl->unit_expert[u]);
+        int bg = __ldcg(&pl->unit_begin[u]);
+        if (cnt < 0 || cnt > kUnitTok || ex < 0 || ex >= args.E || bg < 0 || bg + cnt > nas) {
+          bad = true;
+          cnt = 0;
+          ex = 0;
+          bg = 0;
+        }
+        s_ucnt[u] = (uint8_t)cnt;
+        s_uexp[u] = (uint16_t)ex;
+        s_ubeg[u] = (uint16_t)bg;
+        const int c = cls_of(cnt);
+        T += unit_stages(c, true, H, args.I) + unit_stages(c, false, H, args.I);
+      }
+      for (int i = lane; i < nas; i += 32) {
+        int sl = __ldcg(&pl->assign_slot[i]);
+        if (sl < 0 || sl >= nas) {
+          bad = true;
+          sl = 0;
+        }
+        s_aslot[i] = (uint16_t)sl;
+      }
+      if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(args.status, kStatusOk, kStatusPlan);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) T += __shfl_xor_sync(0xffffffffu, T, off);
+      __syncwarp();
+      sch_B = make_sched(T + S_dn, G, 4);
+      b_known = true;
     };
-    // cursor over the work list (tickets only grow, so it only moves forward).
+    // Cursor over the work list: group (0 shared UP, 1 routed UP, 2 shared
+    // DOWN, 3 routed DOWN), unit, and the list positions
+    // [cur_base, cur_base + cur_size) of its stages.  Tickets only grow, so
+    // the cursor only moves forward.
+    auto g_seg = [&](int g) { return g & 1; };  // 0 shared, 1 routed
+    auto g_up = [&](int g) { return g < 2; };
+    int cur_g = 0, cur_unit = 0, cur_base = 0, cur_size = 0;
+    auto group_units = [&](int g) { return g_seg(g) == 0 ? args.n_su : n_units_r; };
+    auto unit_size = [&](int g, int u) {
+      return g_seg(g) == 0 ? unit_stages(cls_of(su_tokens(u)), g_up(g), H, args.Is)
+                           : unit_stages(cls_of(plan_tokens(u)), g_up(g), H, args.I);
+    };
+    if (args.n_su > 0) cur_size = unit_size(0, 0);
+    auto advance = [&]() {
+      cur_base += cur_size;
+      ++cur_unit;
+      while (cur_unit >= group_units(cur_g)) {
+        cur_unit = 0;
+        if (++cur_g > 3) {  // past the end of the list (positions never get here)
+          cur_size = 1 << 30;
+          return;
+        }
+      }
+      cur_size = unit_size(cur_g, cur_unit);
+    };
     // The current unit's description lives in registers -- lane j also keeps
-    // the token (UP) or slot (DOWN) of the unit's tokens j and j + 32 -- and is
-    // reloaded only when the cursor enters a new unit: with shared memory
-    // taking almost all of the SM, L1 is tiny and per-stage plan loads would
-    // go to L2 every time.
-    bool cur_up = true;
-    int cur_unit = 0;
-    int cur_base = 0, cur_size = n_units > 0 ? unit_stages(0, true) : 0;
-    int u_loaded = -1;
-    bool u_loaded_up = true;
-    int u_ntok = 0, u_cls = 0, u_lw = 0, u_R = 0, u_S = 0, u_begin = 0, u_row0 = 0, u_row1 = 0;
-    int u_out0 = 0, u_out1 = 0;  // flush rows of tokens lane, lane + 32
-    float u_w0 = 1.f, u_w1 = 1.f;
+    // its token's source row (x row for UP, activation row for DOWN), the
+    // row its partial sums go to and its weight -- and is reloaded only when
+    // the cursor enters a new unit: with shared memory taking almost all of
+    // the SM, L1 is tiny and per-stage plan loads would go to L2 every time.
+    int u_seg = -1, u_unit = -1;
+    bool u_up = true;
+    int u_ntok = 0, u_cls = 0, u_lw = 0, u_R = 0, u_S = 0, u_I = 0, u_src = 0, u_dst = 0;
+    float u_w = 1.f;
     const __nv_bfloat16* u_W = nullptr;
     const uint8_t* u_map = nullptr;
     uint32_t q = 0;
-    int ready_panel = -1;  // last (unit, UP panel) seen published
     tk = __shfl_sync(0xffffffffu, tk, 0);
     while (true) {
       int c_beg, c_end;
-      chunk_of(tk, c_beg, c_end);
-      if (c_beg >= T_all || *abort_flag) break;
+      if (tk < sch_A.n_tickets) {
+        sched_range(sch_A, tk, c_beg, c_end);
+      } else {
+        if (!b_known) know_b();
+        const int tr = tk - sch_A.n_tickets;
+        if (tr >= sch_B.n_tickets) break;
+        sched_range(sch_B, tr, c_beg, c_end);
+        c_beg += S_A;
+        c_end += S_A;
+      }
+      if (*abort_flag) break;
       int tk_next = 0;  // next ticket now: its latency overlaps this chunk
       if (lane == 0) tk_next = (int)atomicAdd(&args.queue[0], 1u);
       int piece_start = c_beg;
       bool stop = false;
       for (int t = c_beg; t < c_end; ++t, ++q) {
-        while (t >= cur_base + cur_size) {
-          cur_base += cur_size;
-          if (++cur_unit == n_units) {
-            cur_unit = 0;
-            cur_up = false;
+        while (t >= cur_base + cur_size) advance();
+        const int seg = g_seg(cur_g), unit = cur_unit;  // seg: 0 shared, 1 routed
+        const bool up = g_up(cur_g);
+        if (unit != u_unit || up != u_up || seg != u_seg) {
+          u_seg = seg;
+          u_unit = unit;
+          u_up = up;
+          u_src = u_dst = 0;
+          u_w = 1.f;
+          if (seg == 0) {
+            u_ntok = su_tokens(unit);
+            u_I = args.Is;
+            u_W = up ? args.w13_s : args.w2_s;
+            if (TMAP) u_map = up ? args.maps13_s : args.maps2_s;
+            if (lane < u_ntok) u_src = u_dst = unit * kUnitTok + lane;  // x/h_s (UP), a_s/out (DOWN) rows
+          } else {
+            const int n = s_ucnt[unit];  // sanitised copy of the plan
+            const int expert = s_uexp[unit];
+            const int begin = s_ubeg[unit];
+            u_ntok = n;
+            u_I = args.I;
+            u_W = up ? tab13.p[expert] : tab2.p[expert];
+            if (TMAP) u_map = (up ? args.maps13 : args.maps2) + (size_t)expert * kTensorMapBytes;
+            if (lane < n) {
+              const int slot = s_aslot[begin + lane];
+              const int tok = slot / args.top_k;
+              u_src = up ? tok : slot;  // x row (UP) / a row (DOWN)
+              u_dst = up ? slot : tok;  // h row (UP) / output row (DOWN)
+              if (!up) u_w = __ldcg(&args.plan->assign_w[begin + lane]);
+            }
           }
-          cur_size = unit_stages(cur_unit, cur_up);
-        }
-        const bool up = cur_up;
-        const int unit = cur_unit;
-        if (unit != u_loaded || up != u_loaded_up) {
-          u_loaded = unit;
-          u_loaded_up = up;
-          u_ntok = unit_tokens(unit);
-          u_cls = unit_class(u_ntok);
+          u_cls = cls_of(u_ntok);
           u_lw = class_lw(u_cls);
           u_R = class_rows(u_cls);
-          u_S = unit_panel_stages(u_cls, up, H, I);
-          const int expert = DENSE ? 0 : plan->unit_expert[unit];
-          u_begin = DENSE ? 0 : plan->unit_begin[unit];
-          u_W = up ? (DENSE ? args.w13 : tab13.p[expert]) : (DENSE ? args.w2 : tab2.p[expert]);
-          if (TMAP) u_map = (up ? args.maps13 : args.maps2) + (size_t)(DENSE ? 0 : expert) * kTensorMapBytes;
-          // per token: the row its activations are read from (x row for UP,
-          // a row for DOWN) and the row its partial sums go to (h row for UP,
-          // output row for DOWN) with the routing weight
-          u_row0 = u_row1 = u_out0 = u_out1 = 0;
-          u_w0 = u_w1 = 1.f;
-          if (lane < u_ntok) {
-            const int tk0 = DENSE ? lane : plan->assign_tok[u_begin + lane];
-            const int sl0 = DENSE ? lane : plan->assign_slot[u_begin + lane];
-            u_row0 = up ? tk0 : sl0;
-            u_out0 = up ? sl0 : tk0;
-            if (!DENSE && !up) u_w0 = plan->assign_w[u_begin + lane];
-          }
-          if (lane + 32 < u_ntok) {
-            const int tk1 = DENSE ? lane + 32 : plan->assign_tok[u_begin + lane + 32];
-            const int sl1 = DENSE ? lane + 32 : plan->assign_slot[u_begin + lane + 32];
-            u_row1 = up ? tk1 : sl1;
-            u_out1 = up ? sl1 : tk1;
-            if (!DENSE && !up) u_w1 = plan->assign_w[u_begin + lane + 32];
-          }
+          u_S = unit_panel_stages(u_cls, up, H, u_I);
         }
-        const int ntok = u_ntok, cls = u_cls, lw = u_lw, R = u_R, S = u_S, begin = u_begin;
+        const int ntok = u_ntok, cls = u_cls, lw = u_lw, R = u_R, S = u_S, Iu = u_I;
         const int loc = t - cur_base;
         const int cp = loc / S;
         const int st = loc - cp * S;
@@ -490,33 +623,39 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
         const bool first = (t == piece_start);
         const bool last = (t == c_end - 1 || st == S - 1);
         const int row0 = st * R;
-        const int nrows = min(R, (up ? H : I) - row0);
+        const int nrows = min(R, (up ? H : Iu) - row0);
         // DOWN reads activation rows [row0, row0 + R): wait for the UP panel
         // that produces them (gate columns [p*lw/2, (p+1)*lw/2))
-        const int need_panel = up ? -1 : unit * args.panel_stride + row0 / (lw / 2);
-        if (!up && need_panel != ready_panel) {
-          int ok = 1;
-          if (lane == 0) {
-            uint32_t it = 0;
-            while (ld_acquire_u32(&args.panel_ready[need_panel]) != ready_mark) {
-              if (++it > kSpinLimit || *abort_flag) {
-                atomicCAS(args.status, kStatusOk, kStatusTimeout);
-                *abort_flag = 1;
-                ok = 0;
-                break;
+        if (!up) {
+          const int need_p = row0 / (lw / 2);
+          const int need_panel = unit * (seg == 0 ? args.panel_stride_s : args.panel_stride) + need_p;
+          uint32_t* seen = s_ready + (seg == 0 ? kMaxUnits + unit : unit);
+          if (!((*seen >> need_p) & 1u)) {
+            const unsigned* pr = (seg == 0 ? args.panel_ready_s : args.panel_ready) + need_panel;
+            int ok = 1;
+            if (lane == 0) {
+              uint32_t it = 0;
+              while (ld_acquire_u32(pr) != ready_mark) {
+                if (++it > kSpinLimit || *abort_flag) {
+                  atomicCAS(args.status, kStatusOk, kStatusTimeout);
+                  *abort_flag = 1;
+                  ok = 0;
+                  break;
+                }
+                __nanosleep(64);
               }
-              __nanosleep(64);
+              // the activations were written by other CTAs through the generic
+              // proxy; order them before this CTA's TMA (async proxy) reads
+              asm volatile("fence.proxy.async.global;" ::: "memory");
             }
-            // the activations were written by other CTAs through the generic
-            // proxy; order them before this CTA's TMA (async proxy) reads
-            asm volatile("fence.proxy.async.global;" ::: "memory");
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) {
+              stop = true;
+              break;
+            }
+            if (lane == 0) *seen |= 1u << need_p;
+            __syncwarp();
           }
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) {
-            stop = true;
-            break;
-          }
-          ready_panel = need_panel;
         }
         const int slot = q % NS;
         const uint32_t ph = (q / NS) & 1u;
@@ -527,7 +666,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
           break;
         }
         const int c0 = cp * (up ? lw / 2 : lw);
-        const int w = min(up ? lw / 2 : lw, (up ? I : H) - c0);  // columns per half (UP) or panel (DOWN)
+        const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);  // columns per half (UP) or panel (DOWN)
         const uint32_t wbytes = (uint32_t)w * 2;
         const uint32_t pitch = (uint32_t)lw * 2 + 16, xpitch = (uint32_t)R * 2 + 16;
         // tensor-map path: loads = halves x 16-row blocks x groups of 4 chunks
@@ -540,15 +679,12 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
         uint8_t* sx = sw + kStageWBytes;
         StageHdr& hd = hdr[slot];
         if (lane < ntok) {
-          hd.row[lane] = u_out0;
-          hd.wt[lane] = u_w0;
-        }
-        if (lane + 32 < ntok) {
-          hd.row[lane + 32] = u_out1;
-          hd.wt[lane + 32] = u_w1;
+          hd.row[lane] = u_dst;
+          hd.wt[lane] = u_w;
         }
         if (lane == 0) {
           hd.kind = up ? kKindUp : kKindDown;
+          hd.seg = seg;
           hd.unit = unit;
           hd.cls = cls;
           hd.cp = cp;
@@ -556,13 +692,14 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
           hd.nrows = nrows;
           hd.flags = (first ? kFirst : 0) | (last ? kLast : 0);
           hd.ntok = ntok;
-          hd.begin = begin;
           hd.pstages = t - piece_start + 1;
         }
         __syncwarp();  // every lane's header writes precede lane 0's (releasing) arrive
         if (lane == 0) mbar_arrive_expect_tx(&full[slot], bytes);
         __syncwarp();
-        const __nv_bfloat16* W = u_W;
+        // activations of this lane's token: x row (UP) or a row (DOWN)
+        const void* act = up ? (const void*)(args.x + (size_t)u_src * H + row0)
+                             : (const void*)((seg == 0 ? args.a_s : args.a) + (size_t)u_src * Iu + row0);
         if (TMAP) {
           const int per_half = t_nrb * t_ncg;
           const int rbstride = (lw / kChunkCols) * kChunkTile;
@@ -571,44 +708,21 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
             const int hh = o / per_half, rem = o - hh * per_half;
             const int rb = rem / t_ncg, cg = rem - rb * t_ncg;
             uint8_t* dst = sw + (size_t)rb * rbstride + (size_t)(hh * nch_half + cg * kBoxChunks) * kChunkTile;
-            const int col0 = up ? (hh ? I + c0 : c0) : c0;
+            const int col0 = up ? (hh ? Iu + c0 : c0) : c0;
             tma_load_3d(dst, u_map, 0, row0 + rb * kBoxRows, col0 / kChunkCols + cg * kBoxChunks, &full[slot], pol);
           }
-        }
-        if (TMAP) {
-          // activations only (the weights went above)
-          if (lane < ntok)
-            bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, (up ? (const void*)(args.x + (size_t)u_row0 * H + row0)
-                                                                : (const void*)(args.a + (size_t)u_row0 * I + row0)),
-                                (uint32_t)nrows * 2, &full[slot]);
-          if (lane + 32 < ntok)
-            bulk_copy_g2s_plain(sx + (size_t)(lane + 32) * xpitch,
-                                (up ? (const void*)(args.x + (size_t)u_row1 * H + row0)
-                                    : (const void*)(args.a + (size_t)u_row1 * I + row0)),
-                                (uint32_t)nrows * 2, &full[slot]);
         } else if (up) {
           for (int r = lane; r < nrows; r += 32) {
-            const __nv_bfloat16* src = W + (size_t)(row0 + r) * (2 * I) + c0;
+            const __nv_bfloat16* src = u_W + (size_t)(row0 + r) * (2 * Iu) + c0;
             uint8_t* d = sw + (size_t)r * pitch;
             bulk_copy_g2s(d, src, wbytes, &full[slot], pol);
-            bulk_copy_g2s(d + wbytes, src + I, wbytes, &full[slot], pol);
+            bulk_copy_g2s(d + wbytes, src + Iu, wbytes, &full[slot], pol);
           }
-          if (lane < ntok)
-            bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, args.x + (size_t)u_row0 * H + row0, (uint32_t)nrows * 2,
-                                &full[slot]);
-          if (lane + 32 < ntok)
-            bulk_copy_g2s_plain(sx + (size_t)(lane + 32) * xpitch, args.x + (size_t)u_row1 * H + row0,
-                                (uint32_t)nrows * 2, &full[slot]);
         } else {
           for (int r = lane; r < nrows; r += 32)
-            bulk_copy_g2s(sw + (size_t)r * pitch, W + (size_t)(row0 + r) * H + c0, wbytes, &full[slot], pol);
-          if (lane < ntok)
-            bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, args.a + (size_t)u_row0 * I + row0, (uint32_t)nrows * 2,
-                                &full[slot]);
-          if (lane + 32 < ntok)
-            bulk_copy_g2s_plain(sx + (size_t)(lane + 32) * xpitch, args.a + (size_t)u_row1 * I + row0,
-                                (uint32_t)nrows * 2, &full[slot]);
+            bulk_copy_g2s(sw + (size_t)r * pitch, u_W + (size_t)(row0 + r) * H + c0, wbytes, &full[slot], pol);
         }
+        if (lane < ntok) bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, act, (uint32_t)nrows * 2, &full[slot]);
         if (lane == 0) s_misc[2] = (int)(q + 1);
       }
       if (stop) break;
@@ -625,8 +739,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
     }
   } else {
     // =============================================================== consumers
-    cudaGridDependencySynchronize();
-    const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
+    // (they read nothing the router writes: the stage headers carry it)
     constexpr int NF = acc_frags(KC);
     float acc[NF][4];
     uint32_t q = 0;
@@ -635,13 +748,15 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       const uint32_t ph = (q / NS) & 1u;
       const bool landed = mbar_wait_abortable(&full[slot], ph, args.status, abort_flag);
       // the header stays valid until this warp releases the slot (below,
-      // after any flush that reads its token rows)
+      // once the stage's tensor-core work is done)
       const StageHdr& hd = hdr[slot];
       if (!landed || hd.kind == kKindEnd) break;
       const bool up = hd.kind == kKindUp;
+      const bool sh = hd.seg == 0;
+      const int Iu = sh ? args.Is : args.I;
       const int lw = class_lw(hd.cls);
       const int c0 = hd.cp * (up ? lw / 2 : lw);
-      const int w = min(up ? lw / 2 : lw, (up ? I : H) - c0);
+      const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);
       // local layout of the stage: UP gate [0, w), up [uoff, uoff + w); DOWN [0, w)
       const int uoff = up ? (TMAP ? lw / 2 : w) : 0;
       const int LW = up ? uoff + w : w;
@@ -659,27 +774,32 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       else if constexpr (KC >= 1) {
         if (hd.cls == 1)
           mma_stage<1, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-        else if constexpr (KC >= 2) {
-          if (hd.cls == 2)
-            mma_stage<2, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-          else if constexpr (KC >= 3)
-            mma_stage<3, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-        }
+        else if constexpr (KC >= 2)
+          mma_stage<2, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
       }
-      if (hd.flags & kLast) {
+      const bool piece_end = (hd.flags & kLast) != 0;
+      // What the flush and the SwiGLU fix-up need from the header goes to
+      // registers (lane n keeps token n's row and weight), so the slot can be
+      // handed back to the producer before the flush: its atomics and fence
+      // then overlap the next stages' loads instead of stalling the ring.
+      const int ntok = hd.ntok, cls = hd.cls, cp = hd.cp, unit = hd.unit, pstages = hd.pstages;
+      const int my_row = lane < ntok ? hd.row[lane] : 0;
+      const float my_wt = lane < ntok ? hd.wt[lane] : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);  // release the stage (data and header)
+      ++q;
+      if (piece_end) {
         // ------------------------------------------- flush the piece's sums
+        float* fbase = up ? (sh ? args.h_s : args.h) : args.acc;
+        const size_t ld = up ? 2 * (size_t)Iu : (size_t)H;
         if (!*abort_flag) {
-          if (hd.cls == 0)
-            flush_piece<0, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
+          if (cls == 0)
+            flush_piece<0, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
           else if constexpr (KC >= 1) {
-            if (hd.cls == 1)
-              flush_piece<1, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
-            else if constexpr (KC >= 2) {
-              if (hd.cls == 2)
-                flush_piece<2, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
-              else if constexpr (KC >= 3)
-                flush_piece<3, NF, CW>(acc, args, hd, up, c0, w, uoff, LW, warp, lane);
-            }
+            if (cls == 1)
+              flush_piece<1, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
+            else if constexpr (KC >= 2)
+              flush_piece<2, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
           }
         }
         if (up) {
@@ -689,47 +809,50 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
           // barrier across warps is needed.
           __threadfence();
           __syncwarp();
-          const int panel = hd.unit * args.panel_stride + hd.cp;
-          const unsigned target = (unsigned)unit_panel_stages(hd.cls, true, H, I) * CW;
+          unsigned* pcnt = sh ? args.panel_cnt_s : args.panel_cnt;
+          unsigned* pready = sh ? args.panel_ready_s : args.panel_ready;
+          const int panel = unit * (sh ? args.panel_stride_s : args.panel_stride) + cp;
+          const unsigned target = (unsigned)unit_panel_stages(cls, true, H, Iu) * CW;
           int last = 0;
           if (lane == 0 && !*abort_flag) {
-            const unsigned steps = (unsigned)hd.pstages;
-            const unsigned old = atomicAdd(&args.panel_cnt[panel], steps);
+            const unsigned steps = (unsigned)pstages;
+            const unsigned old = atomicAdd(&pcnt[panel], steps);
             last = (old + steps == target) ? 1 : 0;
           }
           last = __shfl_sync(0xffffffffu, last, 0);
           if (last) {
             __threadfence();
+            float* hb = sh ? args.h_s : args.h;
+            __nv_bfloat16* ab = sh ? args.a_s : args.a;
             const int w4 = w / 4;
-            const int total = hd.ntok * w4;
-            for (int i = lane; i < total; i += 32) {
-              const int n = i / w4;
+            const int total = ntok * w4;
+            for (int i0 = 0; i0 < total; i0 += 32) {  // warp-uniform trip count (shuffles inside)
+              const int i = i0 + lane;
+              const int n = i < total ? i / w4 : 0;
+              const int r = __shfl_sync(0xffffffffu, my_row, n);
+              if (i >= total) continue;
               const int c = c0 + 4 * (i - n * w4);
-              const int slot_id = hd.row[n];
-              float* hg = args.h + (size_t)slot_id * (2 * I) + c;
+              float* hg = hb + (size_t)r * (2 * Iu) + c;
               const float4 g = __ldcg(reinterpret_cast<const float4*>(hg));
-              const float4 u = __ldcg(reinterpret_cast<const float4*>(hg + I));
+              const float4 u = __ldcg(reinterpret_cast<const float4*>(hg + Iu));
               const __nv_bfloat162 lo = __floats2bfloat162_rn(silu_f32(g.x) * u.x, silu_f32(g.y) * u.y);
               const __nv_bfloat162 hi = __floats2bfloat162_rn(silu_f32(g.z) * u.z, silu_f32(g.w) * u.w);
               uint2 pk;
               pk.x = *reinterpret_cast<const uint32_t*>(&lo);
               pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-              *reinterpret_cast<uint2*>(args.a + (size_t)slot_id * I + c) = pk;
+              *reinterpret_cast<uint2*>(ab + (size_t)r * Iu + c) = pk;
               __stcg(reinterpret_cast<float4*>(hg), make_float4(0.f, 0.f, 0.f, 0.f));
-              __stcg(reinterpret_cast<float4*>(hg + I), make_float4(0.f, 0.f, 0.f, 0.f));
+              __stcg(reinterpret_cast<float4*>(hg + Iu), make_float4(0.f, 0.f, 0.f, 0.f));
             }
             __threadfence();
             __syncwarp();
             if (lane == 0) {
-              args.panel_cnt[panel] = 0u;
-              atomicExch(&args.panel_ready[panel], ready_mark);  // publish after the fence above
+              pcnt[panel] = 0u;
+              atomicExch(&pready[panel], ready_mark);  // publish after the fence above
             }
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);  // release the stage (data and header)
-      ++q;
     }
   }
 

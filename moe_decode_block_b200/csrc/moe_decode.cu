@@ -1,14 +1,20 @@
 // moe_decode.cu -- host side of the C ABI declared in include/moe_decode.h.
 //
-// One forward enqueues four kernels:
-//   stream_main: router+top-k+plan, routed experts (UP + SwiGLU + DOWN), [join] combine
-//   stream_aux : shared expert (UP + SwiGLU + DOWN, weight 1), forked after the router
-// The shared expert is forked from stream_main with an event and joined back
-// before the combine (pages: "Hyper Optimizing Kimi K3 in vLLM", section
-// "Recovering time between operators": the shared expert runs on another
-// stream, overlapping routing and the selected experts).  Consecutive kernels
-// on one stream use programmatic dependent launch so the next kernel's CTAs
-// start (and prefetch static weights) while the previous one drains.
+// Two execution plans (pages: "Hyper Optimizing Kimi K3 in vLLM", section
+// "Recovering time between operators": the shared expert overlaps routing,
+// weights are fetched before their consumer starts, the residual add is
+// fused into the producing epilogue, fewer launches per layer):
+//   default (three kernels, stream_main only):
+//     router+top-k+plan; the persistent expert kernel, which streams the
+//     shared expert's up projection before its grid-dependency wait (so it
+//     overlaps the router) and then the routed experts and the shared
+//     expert's down projection; combine + residual.
+//   MOE_FLAG_TWO_STREAM (four kernels, the pages' layout):
+//     stream_main: router, routed experts, [join] combine
+//     stream_aux : shared expert, forked with an event after the router
+// Consecutive kernels on one stream use programmatic dependent launch so the
+// next kernel's CTAs start (and fetch static weights) while the previous one
+// drains.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -54,7 +60,7 @@ bool shapes_valid(const moe_decode_shapes* s) {
   if (s->n_shared != 0 && s->n_shared != 1) return false;
   if (s->n_shared == 1 && (!in(s->shared_inter, 8, 16384) || s->shared_inter % 8)) return false;
   if (!in(s->max_batch, 1, moe::kMaxBatch)) return false;
-  if (s->flags != 0) return false;
+  if ((s->flags & ~MOE_FLAG_TWO_STREAM) != 0) return false;
   return true;
 }
 
@@ -62,6 +68,11 @@ bool shapes_valid(const moe_decode_shapes* s) {
 // experts routed more than kMaxUnitTokens tokens.
 size_t max_units(const moe_decode_shapes* s) {
   return (size_t)s->n_experts + ((size_t)s->max_batch * s->top_k) / moe::kMaxUnitTokens;
+}
+
+// Units of the shared expert for a batch (each holds at most kMaxUnitTokens).
+inline int shared_units(const moe_decode_shapes& s, int batch) {
+  return s.n_shared ? (batch + moe::kMaxUnitTokens - 1) / moe::kMaxUnitTokens : 0;
 }
 
 WorkspaceLayout layout_for(const moe_decode_shapes* s) {
@@ -90,8 +101,9 @@ WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   L.queue = take(4 * 4);
   L.h_s = take(B * 2 * Is * 4);
   L.a_s = take(B * Is * 2);
-  L.panel_cnt_s = take((size_t)ncp_s * 4 + 4);
-  L.panel_ready_s = take((size_t)ncp_s * 4 + 4);
+  const size_t su = (size_t)shared_units(*s, s->max_batch);
+  L.panel_cnt_s = take(su * ncp_s * 4 + 4);
+  L.panel_ready_s = take(su * ncp_s * 4 + 4);
   L.queue_s = take(4 * 4);
   L.acc = take(B * H * 4);
   L.x_stage = take(B * H * 2);
@@ -133,20 +145,22 @@ cudaError_t launch(void (*kern)(KArgs...), int grid, int block, size_t smem, cud
 
 using MlpKernel = void (*)(MmaArgs, ExpertTable, ExpertTable);
 
-// The expert kernel compiled for the largest token class `kc` (0..3) a
+// The expert kernel compiled for the largest token class `kc` (0..2) a
 // launch can see, on the tensor-map or the row-copy path.
-template <bool DENSE, bool TMAP>
+template <bool TMAP>
 MlpKernel pick_mlp_t(int kc) {
   switch (kc) {
-    case 0: return moe::expert_mlp_kernel<DENSE, 0, TMAP>;
-    case 1: return moe::expert_mlp_kernel<DENSE, 1, TMAP>;
-    case 2: return moe::expert_mlp_kernel<DENSE, 2, TMAP>;
-    default: return moe::expert_mlp_kernel<DENSE, 3, TMAP>;
+    case 0: return moe::expert_mlp_kernel<0, TMAP>;
+    case 1: return moe::expert_mlp_kernel<1, TMAP>;
+    default: return moe::expert_mlp_kernel<2, TMAP>;
   }
 }
-template <bool DENSE>
-MlpKernel pick_mlp(int kc, bool tmap) {
-  return tmap ? pick_mlp_t<DENSE, true>(kc) : pick_mlp_t<DENSE, false>(kc);
+MlpKernel pick_mlp(int kc, bool tmap) { return tmap ? pick_mlp_t<true>(kc) : pick_mlp_t<false>(kc); }
+
+// Token class the expert kernel is compiled for at this batch: units hold
+// at most kMaxUnitTokens tokens.
+inline int kernel_class(int batch) {
+  return moe::class_for_tokens(batch < moe::kMaxUnitTokens ? batch : moe::kMaxUnitTokens);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link
@@ -248,9 +262,9 @@ int shared_grid(const moe_decode_ctx* h, int batch) {
   const double E = s.n_experts, k = s.top_k;
   const double distinct = E * (1.0 - std::pow(1.0 - k / E, (double)batch));
   const double routed = distinct * 3.0 * s.hidden * s.inter;
-  const int cls = moe::class_for_tokens(batch);
-  const double slow = cls <= 1 ? 1.3 : (cls == 2 ? 3.0 : 6.0);
-  const double shared = 3.0 * s.hidden * s.shared_inter * slow;
+  const int cls = kernel_class(batch);
+  const double slow = cls <= 1 ? 1.3 : 3.0;
+  const double shared = shared_units(s, batch) * 3.0 * s.hidden * s.shared_inter * slow;
   int g = (int)std::ceil(h->num_sms * shared / (shared + routed));
   const int cap = h->num_sms / 2;
   g = g < 1 ? 1 : (g > cap ? cap : g);
@@ -262,9 +276,7 @@ int set_kernel_attrs(const moe_decode_ctx* h) {
   cudaError_t e;
   for (int kc = 0; kc < moe::kNumClasses; ++kc) {
     for (int tm = 0; tm < 2; ++tm) {
-      e = cudaFuncSetAttribute(pick_mlp<false>(kc, tm), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return fail_cuda(e);
-      e = cudaFuncSetAttribute(pick_mlp<true>(kc, tm), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = cudaFuncSetAttribute(pick_mlp(kc, tm), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return fail_cuda(e);
     }
   }
@@ -332,9 +344,13 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   const uint8_t* maps = h->ws + h->L.maps;
   const size_t mb = moe::kTensorMapBytes;
   int* status = h->at<int>(h->L.status);
-  float* acc = h->at<float>(h->L.acc);
-  const bool fork = s.n_shared && sa != sm;
+  const bool two_stream = (s.flags & MOE_FLAG_TWO_STREAM) != 0;
+  const bool fork = two_stream && s.n_shared && sa != sm;
   const size_t smem = moe::mma_smem_bytes(h->n_stages);
+  const int n_su = shared_units(s, batch);
+  const int kc = kernel_class(batch);
+  const MlpKernel mlp = pick_mlp(kc, h->use_tmap);
+  const int mlp_threads = moe::expert_threads(kc);
 
   auto bail = [&](cudaError_t err) {
     h->dirty = true;
@@ -344,44 +360,37 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     return h->timing ? cudaEventRecord(h->tev[i], st) : cudaSuccess;
   };
 
-  // Shared expert (weight 1, all tokens): on stream_aux, forked after the
-  // router is enqueued so the router's CTAs are dispatched first.  Its grid
-  // is sized to its share of the bytes (the rest of the SMs stream routed
-  // experts), so both finish together instead of contending for every SM.
-  auto launch_shared = [&](cudaStream_t st_sh) -> cudaError_t {
-    MmaArgs ga{};
-    ga.H = s.hidden;
-    ga.I = s.shared_inter;
-    ga.panel_stride = moe::max_up_panels(s.shared_inter);
-    ga.n_stages = h->n_stages;
-    ga.batch = batch;
-    ga.max_units = 1;
-    ga.w13 = static_cast<const __nv_bfloat16*>(shared_w13);
-    ga.w2 = static_cast<const __nv_bfloat16*>(shared_w2);
-    ga.maps13 = maps + 2 * (size_t)s.n_experts * mb;
-    ga.maps2 = maps + (2 * (size_t)s.n_experts + 1) * mb;
-    ga.plan = nullptr;
-    ga.x = static_cast<const __nv_bfloat16*>(x);
-    ga.h = h->at<float>(h->L.h_s);
-    ga.a = h->at<__nv_bfloat16>(h->L.a_s);
-    ga.acc = acc;
-    ga.panel_cnt = h->at<unsigned>(h->L.panel_cnt_s);
-    ga.panel_ready = h->at<unsigned>(h->L.panel_ready_s);
-    ga.queue = h->at<unsigned>(h->L.queue_s);
-    ga.status = status;
-    cudaError_t err = mark(4, st_sh);
-    if (err != cudaSuccess) return err;
-    const int kc_s = moe::class_for_tokens(batch);
-    err = launch(pick_mlp<true>(kc_s, h->use_tmap), shared_grid(h, batch), moe::expert_threads(kc_s), smem,
-                 st_sh, false, ga, *h->tab_none, *h->tab_none);
-    if (err != cudaSuccess) return err;
-    ++kernels;
-    return mark(5, st_sh);
-  };
-  if (fork) {
-    if ((e = cudaEventRecord(h->ev_fork, sm)) != cudaSuccess) return bail(e);
-    if ((e = cudaStreamWaitEvent(sa, h->ev_fork, 0)) != cudaSuccess) return bail(e);
-  }
+  // Arguments common to every expert-kernel launch of this forward.
+  MmaArgs base{};
+  base.H = s.hidden;
+  base.I = s.inter;
+  base.Is = s.n_shared ? s.shared_inter : 0;
+  base.E = s.n_experts;
+  base.top_k = s.top_k;
+  base.n_stages = h->n_stages;
+  base.batch = batch;
+  base.max_units = (int)max_units(&s);
+  base.panel_stride = moe::max_up_panels(s.inter);
+  base.panel_stride_s = s.n_shared ? moe::max_up_panels(s.shared_inter) : 0;
+  base.w13_s = static_cast<const __nv_bfloat16*>(shared_w13);
+  base.w2_s = static_cast<const __nv_bfloat16*>(shared_w2);
+  base.maps13 = maps;
+  base.maps2 = maps + (size_t)s.n_experts * mb;
+  base.maps13_s = maps + 2 * (size_t)s.n_experts * mb;
+  base.maps2_s = maps + (2 * (size_t)s.n_experts + 1) * mb;
+  base.plan = h->at<Plan>(h->L.plan);
+  base.x = static_cast<const __nv_bfloat16*>(x);
+  base.h = h->at<float>(h->L.h);
+  base.a = h->at<__nv_bfloat16>(h->L.a);
+  base.h_s = h->at<float>(h->L.h_s);
+  base.a_s = h->at<__nv_bfloat16>(h->L.a_s);
+  base.acc = h->at<float>(h->L.acc);
+  base.panel_cnt = h->at<unsigned>(h->L.panel_cnt);
+  base.panel_ready = h->at<unsigned>(h->L.panel_ready);
+  base.panel_cnt_s = h->at<unsigned>(h->L.panel_cnt_s);
+  base.panel_ready_s = h->at<unsigned>(h->L.panel_ready_s);
+  base.queue = h->at<unsigned>(h->L.queue);
+  base.status = status;
 
   // Router + top-k + plan.
   RouterArgs ra{};
@@ -400,62 +409,85 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   ra.topk_ids = topk_ids;
   ra.topk_w = topk_w;
   ra.status = status;
-  if ((e = mark(0, sm)) != cudaSuccess) return bail(e);
-  e = launch(pick_router(s.n_experts), ra.G, moe::kRouterThreads,
-             moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra);
-  if (e != cudaSuccess) return bail(e);
-  ++kernels;
-  if ((e = mark(1, sm)) != cudaSuccess) return bail(e);
-  if (fork) {
-    if ((e = launch_shared(sa)) != cudaSuccess) return bail(e);
-    if ((e = cudaEventRecord(h->ev_join, sa)) != cudaSuccess) return bail(e);
-  }
+  auto launch_router = [&]() -> cudaError_t {
+    cudaError_t err = mark(0, sm);
+    if (err != cudaSuccess) return err;
+    err = launch(pick_router(s.n_experts), ra.G, moe::kRouterThreads,
+                 moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra);
+    if (err != cudaSuccess) return err;
+    ++kernels;
+    return mark(1, sm);
+  };
 
-  // Routed experts: UP + SwiGLU + DOWN in one persistent launch.
-  MmaArgs ma{};
-  ma.H = s.hidden;
-  ma.I = s.inter;
-  ma.panel_stride = moe::max_up_panels(s.inter);
-  ma.n_stages = h->n_stages;
-  ma.batch = batch;
-  ma.max_units = (int)max_units(&s);
-  ma.plan = h->at<Plan>(h->L.plan);
-  ma.maps13 = maps;
-  ma.maps2 = maps + (size_t)s.n_experts * mb;
-  ma.x = static_cast<const __nv_bfloat16*>(x);
-  ma.h = h->at<float>(h->L.h);
-  ma.a = h->at<__nv_bfloat16>(h->L.a);
-  ma.acc = acc;
-  ma.panel_cnt = h->at<unsigned>(h->L.panel_cnt);
-  ma.panel_ready = h->at<unsigned>(h->L.panel_ready);
-  ma.queue = h->at<unsigned>(h->L.queue);
-  ma.status = status;
-  int g_routed = h->grid_routed;
-  if (fork && h->grid_routed_auto) {
-    g_routed = h->num_sms - shared_grid(h, batch);
-    if (g_routed < 1) g_routed = 1;
-  }
-  // a unit holds at most kMaxUnitTokens tokens (larger experts are split)
-  const int routed_kc = moe::class_for_tokens(batch < moe::kMaxUnitTokens ? batch : moe::kMaxUnitTokens);
-  e = launch(pick_mlp<false>(routed_kc, h->use_tmap), g_routed, moe::expert_threads(routed_kc), smem, sm, true, ma,
-             *h->tab13,
-             *h->tab2);
-  if (e != cudaSuccess) return bail(e);
-  ++kernels;
-  if ((e = mark(2, sm)) != cudaSuccess) return bail(e);
-  if (s.n_shared && !fork) {
-    if ((e = launch_shared(sm)) != cudaSuccess) return bail(e);
-  }
+  auto launch_combine = [&](bool pdl) -> cudaError_t {
+    const int nvec = batch * s.hidden / 8;
+    cudaError_t err = launch(moe::combine_residual_kernel, ceil_div(nvec, 256), 256, 0, sm, pdl,
+                             static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec);
+    if (err != cudaSuccess) return err;
+    ++kernels;
+    return mark(3, sm);
+  };
 
-  if (fork) {
-    if ((e = cudaStreamWaitEvent(sm, h->ev_join, 0)) != cudaSuccess) return bail(e);
+  if (!two_stream) {
+    // -------------------------------------------- default: three kernels
+    MmaArgs ma = base;
+    ma.n_su = n_su;
+    ma.has_routed = 1;
+    if ((e = launch_router()) != cudaSuccess) return bail(e);
+    if ((e = mark(4, sm)) != cudaSuccess) return bail(e);
+    e = launch(mlp, h->grid_routed, mlp_threads, smem, sm, true, ma, *h->tab13, *h->tab2);
+    if (e != cudaSuccess) return bail(e);
+    ++kernels;
+    if ((e = mark(2, sm)) != cudaSuccess || (e = mark(5, sm)) != cudaSuccess) return bail(e);
+    if ((e = launch_combine(true)) != cudaSuccess) return bail(e);
+  } else {
+    // ------------------------------------ MOE_FLAG_TWO_STREAM: four kernels
+    // Shared expert (weight 1, all tokens): on stream_aux, forked after the
+    // router is enqueued so the router's CTAs are dispatched first.  Its grid
+    // is sized to its share of the bytes (the rest of the SMs stream routed
+    // experts), so both finish together instead of contending for every SM.
+    auto launch_shared = [&](cudaStream_t st_sh) -> cudaError_t {
+      MmaArgs ga = base;
+      ga.n_su = n_su;
+      ga.has_routed = 0;
+      ga.queue = h->at<unsigned>(h->L.queue_s);
+      cudaError_t err = mark(4, st_sh);
+      if (err != cudaSuccess) return err;
+      err = launch(mlp, shared_grid(h, batch), mlp_threads, smem, st_sh, false, ga, *h->tab_none, *h->tab_none);
+      if (err != cudaSuccess) return err;
+      ++kernels;
+      return mark(5, st_sh);
+    };
+    if (fork) {
+      if ((e = cudaEventRecord(h->ev_fork, sm)) != cudaSuccess) return bail(e);
+      if ((e = cudaStreamWaitEvent(sa, h->ev_fork, 0)) != cudaSuccess) return bail(e);
+    }
+    if ((e = launch_router()) != cudaSuccess) return bail(e);
+    if (fork) {
+      if ((e = launch_shared(sa)) != cudaSuccess) return bail(e);
+      if ((e = cudaEventRecord(h->ev_join, sa)) != cudaSuccess) return bail(e);
+    }
+    // Routed experts: UP + SwiGLU + DOWN in one persistent launch.
+    MmaArgs ma = base;
+    ma.n_su = 0;
+    ma.has_routed = 1;
+    int g_routed = h->grid_routed;
+    if (fork && h->grid_routed_auto) {
+      g_routed = h->num_sms - shared_grid(h, batch);
+      if (g_routed < 1) g_routed = 1;
+    }
+    e = launch(mlp, g_routed, mlp_threads, smem, sm, true, ma, *h->tab13, *h->tab2);
+    if (e != cudaSuccess) return bail(e);
+    ++kernels;
+    if ((e = mark(2, sm)) != cudaSuccess) return bail(e);
+    if (s.n_shared && !fork) {
+      if ((e = launch_shared(sm)) != cudaSuccess) return bail(e);
+    }
+    if (fork) {
+      if ((e = cudaStreamWaitEvent(sm, h->ev_join, 0)) != cudaSuccess) return bail(e);
+    }
+    if ((e = launch_combine(!fork)) != cudaSuccess) return bail(e);
   }
-  const int nvec = batch * s.hidden / 8;
-  e = launch(moe::combine_residual_kernel, ceil_div(nvec, 256), 256, 0, sm, !fork,
-             static_cast<const __nv_bfloat16*>(x), acc, static_cast<__nv_bfloat16*>(out), nvec);
-  if (e != cudaSuccess) return bail(e);
-  ++kernels;
-  if ((e = mark(3, sm)) != cudaSuccess) return bail(e);
 
   h->stats.forwards += 1;
   h->stats.kernels_launched += (uint64_t)kernels;

@@ -294,6 +294,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
     a.plan->n_active = ftot;
     if (ctot != nas) atomicCAS(a.status, kStatusOk, kStatusPlan);
   }
+
   __syncthreads();
   // Assignment (t, j) goes to offset[e] + #{t' < t : e in ids[t']} (ids of one
   // token are distinct, so this orders each expert's assignments by token).

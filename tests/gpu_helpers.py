@@ -39,11 +39,19 @@ def margin_x(batch, hidden, wts, k, seed=0, device="cuda", min_gap=MIN_MARGIN):
 class Run:
     """Device buffers and one handle for a block shape."""
 
-    def __init__(self, shape: synth.BlockShape, wts, max_batch=64):
+    def __init__(self, shape: synth.BlockShape, wts, max_batch=64, two_stream=False):
         self.s = shape
         self.wts = wts
         self.blk = MoEDecode(shape.hidden, shape.n_experts, shape.top_k, shape.inter, shape.shared_inter,
-                             n_shared=shape.n_shared, max_batch=max_batch, router_bias=wts.router_bias)
+                             n_shared=shape.n_shared, max_batch=max_batch, router_bias=wts.router_bias,
+                             two_stream=two_stream)
+
+    def kernels_per_forward(self):
+        """Kernels one forward enqueues: router, expert kernel, combine by default;
+        router, routed experts, [shared expert], combine with two streams."""
+        if self.blk.two_stream:
+            return 4 if self.s.n_shared else 3
+        return 3
 
     def forward(self, x, stream_aux=None, w13=None, w2=None):
         B = x.shape[0]

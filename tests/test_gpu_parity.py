@@ -1,7 +1,10 @@
 """CUDA path vs the fp64 oracle on a B200, through the C ABI.
 
 Bar: expert ids exact, renormalised weights within 1e-5, outputs within
-2e-2 * rms(oracle out).  Inputs are seeded and synthetic (weights ~ N(0,0.02),
+2e-2 * rms(oracle out).  Both execution plans are covered: the default one
+(router kernel + one expert kernel with the shared expert, routed experts and
+combine) and the two-stream one (shared expert on the aux stream, separate
+combine kernel).  Inputs are seeded and synthetic (weights ~ N(0,0.02),
 x ~ N(0,1), bf16) with a top-k logit margin >= 1e-3.  Tiny shapes are
 compared element by element for every token; full-size shapes compare the
 ids/weights of every token and the outputs of sampled tokens.
@@ -16,10 +19,13 @@ from gpu_helpers import Run, margin_x, oracle_check
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def tiny():
+PLANS = ["default", "two_stream"]
+
+
+@pytest.fixture(scope="module", params=PLANS)
+def tiny(request):
     wts = synth.make_weights(synth.TINY, seed=0, device="cuda")
-    return Run(synth.TINY, wts, max_batch=64)
+    return Run(synth.TINY, wts, max_batch=64, two_stream=request.param == "two_stream")
 
 
 @pytest.fixture(scope="module")
@@ -40,7 +46,7 @@ def test_tiny_every_element(tiny, B):
     out, ids, w = tiny.forward(x)
     oracle_check(tiny.wts, synth.TINY.top_k, x, out, ids, w)
     st = tiny.blk.stats()
-    assert st["last_kernels"] == 4
+    assert st["last_kernels"] == tiny.kernels_per_forward()
     assert st["last_token_tiles"] == (min(B, 32) + 7) // 8
     assert tiny.blk.status() == MOE_OK
 
@@ -51,24 +57,28 @@ def test_tiny_config_seed0(tiny):
     oracle_check(tiny.wts, synth.TINY.top_k, x, out, ids, w)
 
 
-def test_tiny_top1_and_no_shared():
+@pytest.mark.parametrize("plan", PLANS)
+def test_tiny_top1_and_no_shared(plan):
     s = synth.BlockShape(hidden=256, n_experts=16, top_k=1, inter=128, shared_inter=0, n_shared=0)
     wts = synth.make_weights(s, seed=3, device="cuda")
-    run = Run(s, wts, max_batch=8)
+    run = Run(s, wts, max_batch=8, two_stream=plan == "two_stream")
     x = margin_x(8, s.hidden, wts, 1, seed=3)
     out, ids, w = run.forward(x)
     assert torch.all(w == 1.0)
     oracle_check(wts, 1, x, out, ids, w)
-    assert run.blk.stats()["last_kernels"] == 3
+    assert run.blk.stats()["last_kernels"] == run.kernels_per_forward()
 
 
-def test_tiny_odd_shapes_several_panels_and_ragged_steps():
+@pytest.mark.parametrize("plan", PLANS)
+def test_tiny_odd_shapes_several_panels_and_ragged_steps(plan):
     # inter 2056 -> two UP panels (gate/up pairs) with a ragged last panel;
-    # hidden 4104 -> two DOWN panels; K not a multiple of 64 -> ragged steps
+    # hidden 4104 -> two DOWN panels and a ragged last 512-column combine
+    # block; K not a multiple of 64 -> row-copy path, ragged steps; batch 40
+    # -> two shared-expert units and a split routed unit
     s = synth.BlockShape(hidden=4104, n_experts=24, top_k=3, inter=2056, shared_inter=136, n_shared=1)
     wts = synth.make_weights(s, seed=4, device="cuda")
-    run = Run(s, wts, max_batch=16)
-    for B in (1, 6, 16):
+    run = Run(s, wts, max_batch=40, two_stream=plan == "two_stream")
+    for B in (1, 6, 16, 40):
         x = margin_x(B, s.hidden, wts, s.top_k, seed=40 + B)
         out, ids, w = run.forward(x)
         oracle_check(wts, s.top_k, x, out, ids, w)
@@ -236,3 +246,17 @@ def test_graph_replay_alternating_inputs_full_b8(full):
     xa = margin_x(8, synth.FULL.hidden, full.wts, 8, seed=11)
     xb = margin_x(8, synth.FULL.hidden, full.wts, 8, seed=12)
     _graph_alternating(full, xa, xb, replays=5)
+
+
+@pytest.mark.parametrize("B", [1, 8, 40])
+def test_full_size_two_stream_plan(full, B):
+    run = Run(synth.FULL, full.wts, max_batch=64, two_stream=True)
+    try:
+        x = margin_x(B, synth.FULL.hidden, full.wts, synth.FULL.top_k, seed=200 + B)
+        out, ids, w = run.forward(x)
+        rows = np.unique(np.linspace(0, B - 1, min(B, 4)).astype(int))
+        oracle_check(full.wts, synth.FULL.top_k, x, out, ids, w, rows=rows)
+        assert run.blk.stats()["last_kernels"] == 4
+        assert run.blk.status() == MOE_OK
+    finally:
+        run.blk.close()
