@@ -154,6 +154,24 @@ def bytes_per_step(shape, ids, batch: int) -> tuple[int, int]:
     return distinct * shape.expert_bytes() + shape.shared_bytes() + shape.router_bytes() + act, distinct
 
 
+def aggregate_over_ranks(total_ms: float, bytes_per_step: float, steps: int, device, world: int):
+    """Whole-job throughput of independent replicas: bytes summed over ranks,
+    time = the slowest rank's device time (all_reduce MAX).  Returns
+    (value GB/s, max_total_ms, all_bytes).  Collective calls are the same on
+    every rank, in the same order."""
+    import torch
+    if world > 1:
+        t = torch.tensor([float(total_ms)], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+        bt = torch.tensor([float(bytes_per_step)], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(bt)
+        all_bytes = float(bt.item()) * steps
+    else:
+        all_bytes = float(bytes_per_step) * steps
+    return all_bytes / (total_ms / 1e3) / 1e9, total_ms, all_bytes
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -348,18 +366,8 @@ def run_ours(args):
         torch.distributed.barrier()
     clocks = sampler.stop()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    total_ms = float(sum(step_ms))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-        bt = torch.tensor([float(bstep)], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(bt)
-        all_bytes = float(bt.item()) * args.steps
-    else:
-        all_bytes = float(bstep) * args.steps
+    value, total_ms, all_bytes = aggregate_over_ranks(float(sum(step_ms)), bstep, args.steps, dev, world)
     ms_per_step = total_ms / args.steps
-    value = all_bytes / (total_ms / 1e3) / 1e9
 
     # ---- per-kernel breakdown (eager forwards with timing events)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
