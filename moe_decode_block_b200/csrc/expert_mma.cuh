@@ -196,10 +196,13 @@ __host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int
   return unit_panels(cls, up, H, I) * unit_panel_stages(cls, up, H, I);
 }
 
-// Ticket schedule over a segment of T stages for a grid of G CTAs: 3/4 of
-// the list in chunks of c_big = T / (div * G), then 3/16 in chunks of
-// c_big / 4, then single stages (make_sched); or one round of at most G
-// chunks of max(1, T / G) stages plus the remainder (make_round).
+// Ticket schedule over a segment of T stages for a grid of G CTAs
+// (make_sched): chunks of c_big = T / (div * G) stages (at most kMaxChunk),
+// then about three chunks of c_big / 4 per CTA, then the last 2G stages one
+// at a time -- the tail that balances the end is bounded in stages, not a
+// fraction of the list, because every chunk ends in a flush of the
+// consumers' partial sums.  make_round: one round of at most G chunks of
+// max(1, T / G) stages plus the remainder.
 struct Sched {
   int T, c_big, c_mid, n_big, n_mid, T1, T2, n_tickets;
 };
@@ -223,9 +226,13 @@ __device__ __forceinline__ Sched make_sched(int T, int G, int div) {
   c = c < 1 ? 1 : (c > kMaxChunk ? kMaxChunk : c);
   s.c_big = c;
   s.c_mid = c / 4 < 1 ? 1 : c / 4;
-  s.n_big = (T / 4 * 3) / c;
+  const int singles = T < 2 * G ? T : 2 * G;
+  const int mid_max = 3 * G * s.c_mid;
+  const int rest = T - singles;
+  const int mid = rest < mid_max ? rest : mid_max;
+  s.n_big = (rest - mid) / c;
   s.T1 = s.n_big * c;
-  s.n_mid = ((T - s.T1) / 4 * 3) / s.c_mid;
+  s.n_mid = (T - singles - s.T1) / s.c_mid;
   s.T2 = s.T1 + s.n_mid * s.c_mid;
   s.n_tickets = s.n_big + s.n_mid + (T - s.T2);
   return s;
@@ -349,13 +356,16 @@ __device__ __forceinline__ int local_to_col(int l, bool up, int c0, int w, int u
   return -1;
 }
 
-// Flush this warp's partial sums of a piece (class C) with fp32 atomics into
-// rows base + row(n) * ld, where lane n of the warp holds row(n) in my_row and
-// the weight in my_wt (copied from the stage header, so the stage's slot can
-// be handed back before the flush).  An m-tile's C fragment spreads 16
-// columns of a token over 8 lanes; shuffles gather each run of 4 columns into
-// one lane, so every 16 bytes take one vector atomic instead of four scalar
-// ones.
+// Flush this warp's partial sums of a piece (class C) with fp32 reductions
+// into rows base + row(n) * ld, where lane n of the warp holds row(n) in my_row
+// and the weight in my_wt (copied from the stage header, so the stage's slot
+// can be handed back before the flush).  A lane's C fragment holds columns
+// gid and gid + 8 of an m-tile for tokens 2*tig and 2*tig + 1 of an n-tile;
+// each value goes out as one scalar reduction (red, no return value).  Only
+// token slots that exist are visited, so a one-token piece costs MT x 2
+// reductions per lane of one quad.  (Gathering runs of 4 columns into one
+// lane with shuffles for vector reductions measured slower: the shuffles
+// cost more issue slots than the reductions they save.)
 template <int C, int NF, int CW>
 __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], float* base, size_t ld, int my_row,
                                             float my_wt, int ntok, bool up, int c0, int w, int uoff, int LW, int I,
@@ -370,35 +380,20 @@ __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], float* ba
     if (nt >= ntiles) break;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int n = nt * 8 + tig * 2 + e;  // this lane's token (same for its tig group)
-      const bool valid = n < ntok;
+      if (nt * 8 + e >= ntok) break;       // no lane holds a token here (warp-uniform)
+      const int n = nt * 8 + tig * 2 + e;  // this lane's token
       const int r = __shfl_sync(0xffffffffu, my_row, n);
       const float wr = __shfl_sync(0xffffffffu, my_wt, n);
-      float* row = nullptr;
-      float wt = 1.f;
-      if (valid) {
-        row = base + (size_t)r * ld;
-        wt = up ? 1.f : wr;
-      }
+      if (n < ntok) {
+        float* row = base + (size_t)r * ld;
+        const float wt = up ? 1.f : wr;
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        if (m0 + mt * 16 >= LW) break;
-        const float v_lo = acc[mt * NT + nt][e];      // column gid
-        const float v_hi = acc[mt * NT + nt][2 + e];  // column gid + 8
-        // lane with gid < 4 collects columns 4*gid .. 4*gid + 3 of its token
-        float o[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = 4 * (gid & 3) + j;
-          const int src = ((c & 7) << 2) | tig;
-          const float a = __shfl_sync(0xffffffffu, v_lo, src);
-          const float b = __shfl_sync(0xffffffffu, v_hi, src);
-          o[j] = c < 8 ? a : b;
-        }
-        if (valid && gid < 4) {
-          const int col = local_to_col(m0 + mt * 16 + 4 * gid, up, c0, w, uoff, I);
-          if (col >= 0)
-            atomicAdd(reinterpret_cast<float4*>(row + col), make_float4(wt * o[0], wt * o[1], wt * o[2], wt * o[3]));
+        for (int mt = 0; mt < MT; ++mt) {
+          if (m0 + mt * 16 >= LW) break;
+          const int lo = local_to_col(m0 + mt * 16 + gid, up, c0, w, uoff, I);
+          const int hi = local_to_col(m0 + mt * 16 + gid + 8, up, c0, w, uoff, I);
+          if (lo >= 0) red_add(row + lo, wt * acc[mt * NT + nt][e]);
+          if (hi >= 0) red_add(row + hi, wt * acc[mt * NT + nt][2 + e]);
         }
       }
     }

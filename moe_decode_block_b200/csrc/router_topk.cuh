@@ -14,7 +14,7 @@
 //     under programmatic dependent launch is safe); x is read only after it.
 //   * Each thread owns a pair of expert columns and accumulates the partial
 //     logits of every token over the slab in fp32; partials are reduced into
-//     a global fp32 [B, E] buffer with vector atomics.
+//     a global fp32 [B, E] buffer with vector reductions (red, no return).
 //   * The last CTA to finish (ticket counter) reads the logits, adds the
 //     optional bias, selects the top k per token with warp argmax rounds,
 //     computes the renormalised weights, writes topk_ids/topk_w, builds the
@@ -163,8 +163,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           if (j < nt)
-            atomicAdd(reinterpret_cast<float2*>(a.logits + (size_t)(t0 + j) * E) + p,
-                      make_float2(acc[j][0], acc[j][1]));
+            red_add_v2(a.logits + (size_t)(t0 + j) * E + 2 * p, acc[j][0], acc[j][1]);
       }
     }
     __syncthreads();
