@@ -43,7 +43,7 @@ using moe::RouterArgs;
 thread_local int g_last_cuda_error = 0;
 
 struct WorkspaceLayout {
-  size_t status, ticket, logits, plan, h, a, panel_cnt, panel_ready, queue, h_s, a_s, panel_cnt_s, panel_ready_s,
+  size_t status, ticket, router_epoch, logits, plan, h, a, panel_cnt, panel_ready, queue, h_s, a_s, panel_cnt_s, panel_ready_s,
       queue_s, acc, x_stage, out_stage, ids_stage, w_stage, maps, total;
 };
 
@@ -91,7 +91,8 @@ WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   };
   L.status = take(sizeof(int));
   L.ticket = take(sizeof(unsigned));
-  L.logits = take(B * E * 4);
+  L.router_epoch = take(sizeof(unsigned));
+  L.logits = take(2 * B * E * 4);  // two buffers, used alternately by the router
   L.plan = take(sizeof(Plan));
   L.h = take(B * k * 2 * I * 4);
   L.a = take(B * k * I * 2);
@@ -404,6 +405,8 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   ra.G = router_grid(h, batch);
   ra.chunk_rows = h->router_chunk_rows;
   ra.logits = h->at<float>(h->L.logits);
+  ra.logits_stride = s.max_batch * s.n_experts;
+  ra.epoch = h->at<unsigned>(h->L.router_epoch);
   ra.ticket = h->at<unsigned>(h->L.ticket);
   ra.plan = h->at<Plan>(h->L.plan);
   ra.topk_ids = topk_ids;

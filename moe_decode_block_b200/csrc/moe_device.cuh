@@ -42,8 +42,7 @@ struct Plan {
   int unit_expert[kMaxUnits];
   int unit_begin[kMaxUnits];
   int unit_count[kMaxUnits];
-  int assign_tok[kMaxAssign];   // token index b
-  int assign_slot[kMaxAssign];  // b * top_k + j (row of the per-assignment buffers)
+  int assign_slot[kMaxAssign];  // b * top_k + j: token b = slot / top_k, row of the per-assignment buffers
   float assign_w[kMaxAssign];   // renormalised routing weight
 };
 

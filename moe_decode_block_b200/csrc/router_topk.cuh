@@ -15,11 +15,18 @@
 //   * Each thread owns a pair of expert columns and accumulates the partial
 //     logits of every token over the slab in fp32; partials are reduced into
 //     a global fp32 [B, E] buffer with vector reductions (red, no return).
-//   * The last CTA to finish (ticket counter) reads the logits, adds the
-//     optional bias, selects the top k per token with warp argmax rounds,
-//     computes the renormalised weights, writes topk_ids/topk_w, builds the
-//     bucketed plan (experts ascending, assignments sorted by token) and
-//     returns the logits buffer and the ticket to zero for the next call.
+//   * The last CTA to finish (ticket counter) stages the logits in shared
+//     memory (one batched load per group of tokens), adds the optional bias,
+//     selects the top k per token with warp argmax rounds, computes the
+//     renormalised weights, writes topk_ids/topk_w, builds the bucketed plan
+//     (experts ascending, assignments sorted by token) and returns the ticket
+//     to zero for the next call.
+//   * Zeroing the logits for the next call is spread over all CTAs: with two
+//     buffers used alternately (parity of a launch counter), each CTA clears
+//     a slice of the buffer the next launch will use while it runs its GEMV.
+//     The last CTA runs while the expert kernel already streams weights at
+//     full HBM bandwidth, so every global access it makes queues behind that
+//     traffic: it reads the logits once and writes only the results.
 #pragma once
 
 #include "moe_device.cuh"
@@ -33,7 +40,11 @@ struct RouterArgs {
   int B, H, E, k;
   int G;                        // grid size
   int chunk_rows;               // rows of router_w staged per bulk copy
-  float* logits;                // [B, E] fp32 accumulators, zero between calls
+  float* logits;                // fp32 accumulators [B, E]; see logits_stride
+  int logits_stride;            // 0: one buffer, zero between calls (the last CTA re-zeroes it);
+                                // > 0: two buffers logits and logits + stride (>= B * E floats,
+                                // a multiple of 4), used by launch parity, the unused one zero
+  unsigned* epoch;              // launch counter choosing the buffer (logits_stride > 0)
   unsigned* ticket;             // zero between calls
   Plan* plan;
   int32_t* topk_ids;            // [B, k]
@@ -44,10 +55,16 @@ struct RouterArgs {
 // Tokens padded to a multiple of 8 (x is staged token-contiguous per row).
 __host__ __device__ inline int router_bpad(int B) { return (B + 7) / 8 * 8; }
 
+// Tokens whose logits the last CTA stages in shared memory at once.
+__host__ __device__ inline int router_stage_tokens(int B, int E) {
+  const int tb = 16384 / E;  // 64 KB of fp32 logits
+  return B < tb ? B : (tb < 1 ? 1 : tb);
+}
+
 // Shared memory needed by router_topk_kernel for these sizes.
 __host__ __device__ inline size_t router_smem_bytes(int B, int E, int chunk_rows) {
   size_t gemv = (size_t)chunk_rows * E * 2 + (size_t)router_bpad(B) * chunk_rows * 4;
-  size_t topk = (size_t)kMaxAssign * 8 + (size_t)E * 16 + 64;
+  size_t topk = (size_t)kMaxAssign * 8 + (size_t)E * 16 + 64 + ((size_t)router_stage_tokens(B, E) + 1) * E * 4;
   gemv = (gemv + 15) / 16 * 16;
   return gemv > topk ? gemv : topk;
 }
@@ -61,6 +78,77 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
     if (v2 > v || (v2 == v && i2 < i)) {
       v = v2;
       i = i2;
+    }
+  }
+}
+
+// (value, id) order of the selection: larger logit first, equal logits to the
+// smaller expert id.
+__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+// Top-8 of one token's logits by one warp: lg (shared memory) holds the E
+// logits, bias the per-expert bias; every lane ends with the 8 best
+// (value, id) pairs sorted in selection order.  Each lane first keeps its own
+// best 8 (experts lane + 32 i) in a sorted list (insertion), then five
+// butterfly levels merge lists between lanes l and l ^ off: the element-wise
+// better of list A and reversed list B is a bitonic sequence holding the 8
+// best of both, which a 3-stage bitonic network sorts.  The loops over
+// experts and levels are kept rolled: this runs once per call in one CTA
+// while the expert kernel saturates the memory system, so a long straight
+// line of code would pay for instruction fetches.
+__device__ __forceinline__ void warp_top8(const float* lg, const float* bias, int E, int lane, float (&tv)[8],
+                                          int (&ti)[8]) {
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    tv[r] = -INFINITY;
+    ti[r] = 0x7fffffff;  // after every real expert on ties
+  }
+#pragma unroll 1
+  for (int e = lane; e < E; e += 32) {
+    float cv = lg[e] + bias[e];
+    int ci = e;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const bool sw = ranks_before(cv, ci, tv[r], ti[r]);
+      const float sv = tv[r];
+      const int si = ti[r];
+      tv[r] = sw ? cv : sv;
+      ti[r] = sw ? ci : si;
+      cv = sw ? sv : cv;
+      ci = sw ? si : ci;
+    }
+  }
+#pragma unroll 1
+  for (int off = 1; off < 32; off <<= 1) {
+    float pv[8];
+    int pi[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      pv[r] = __shfl_xor_sync(0xffffffffu, tv[r], off);
+      pi[r] = __shfl_xor_sync(0xffffffffu, ti[r], off);
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const bool sw = ranks_before(pv[7 - r], pi[7 - r], tv[r], ti[r]);
+      tv[r] = sw ? pv[7 - r] : tv[r];
+      ti[r] = sw ? pi[7 - r] : ti[r];
+    }
+#pragma unroll
+    for (int d = 4; d > 0; d >>= 1) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if ((r & d) == 0) {
+          const bool sw = ranks_before(tv[r + d], ti[r + d], tv[r], ti[r]);
+          const float a0 = tv[r], a1 = tv[r + d];
+          const int i0 = ti[r], i1 = ti[r + d];
+          tv[r] = sw ? a1 : a0;
+          ti[r] = sw ? i1 : i0;
+          tv[r + d] = sw ? a0 : a1;
+          ti[r + d] = sw ? i0 : i1;
+        }
+      }
     }
   }
 }
@@ -127,6 +215,17 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   cudaGridDependencySynchronize();
   cudaTriggerProgrammaticLaunchCompletion();
 
+  // this launch's logits buffer; clear this CTA's slice of the other one
+  float* lg_buf = a.logits;
+  if (a.logits_stride > 0) {
+    const unsigned par = __ldcg(a.epoch) & 1u;
+    lg_buf = a.logits + (size_t)par * a.logits_stride;
+    float4* other = reinterpret_cast<float4*>(a.logits + (size_t)(par ^ 1u) * a.logits_stride);
+    const int n4 = a.logits_stride / 4;
+    const int c0 = (int)((long long)n4 * blockIdx.x / a.G), c1 = (int)((long long)n4 * (blockIdx.x + 1) / a.G);
+    for (int i = c0 + tid; i < c1; i += kRouterThreads) __stcg(other + i, make_float4(0.f, 0.f, 0.f, 0.f));
+  }
+
   uint32_t phase = 0;
   const int npairs = E / 2;
   const int bp = router_bpad(B);
@@ -163,7 +262,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
 #pragma unroll
         for (int j = 0; j < 8; ++j)
           if (j < nt)
-            red_add_v2(a.logits + (size_t)(t0 + j) * E + 2 * p, acc[j][0], acc[j][1]);
+            red_add_v2(lg_buf + (size_t)(t0 + j) * E + 2 * p, acc[j][0], acc[j][1]);
       }
     }
     __syncthreads();
@@ -189,18 +288,46 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   int* s_off = s_cnt + E;                                 // [E]
   int* s_act = s_off + E;                                 // [E] active index or -1
 
+  float* s_bias = reinterpret_cast<float*>(s_act + E);  // [E] (16-byte aligned: E % 8 == 0)
+  float* s_lg = s_bias + E;                                 // [TB, E]
+  for (int e = tid; e < E; e += kRouterThreads) s_bias[e] = a.bias ? a.bias[e] : 0.f;
   const int nv = (E + 31) / 32;
-  for (int t = warp; t < B; t += kRouterThreads / 32) {
-    float* lg = a.logits + (size_t)t * E;
+  const int TB = router_stage_tokens(B, E);
+  for (int tb0 = 0; tb0 < B; tb0 += TB) {
+    const int ntb = min(TB, B - tb0);
+    {
+      // one batched load of ntb rows of logits (8 float4 in flight per thread)
+      float4* src = reinterpret_cast<float4*>(lg_buf + (size_t)tb0 * E);
+      float4* dst = reinterpret_cast<float4*>(s_lg);
+      const int n4 = ntb * E / 4;
+      for (int i0 = 0; i0 < n4; i0 += 8 * kRouterThreads) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kRouterThreads + tid;
+          if (i < n4) v[u] = __ldcg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * kRouterThreads + tid;
+          if (i < n4) {
+            dst[i] = v[u];
+            if (a.logits_stride == 0) __stcg(src + i, make_float4(0.f, 0.f, 0.f, 0.f));
+          }
+        }
+      }
+    }
+    __syncthreads();
+  for (int t = tb0 + warp; t < tb0 + ntb; t += kRouterThreads / 32) {
+    const float* lg = s_lg + (size_t)(t - tb0) * E;
     float v[NV];
     uint32_t taken = 0;
+    if (k > 8) {
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const int e = lane + 32 * i;
-      v[i] = -INFINITY;
-      if (i < nv && e < E) {
-        v[i] = __ldcg(lg + e) + (a.bias ? a.bias[e] : 0.f);
-        __stcg(lg + e, 0.f);
+      for (int i = 0; i < NV; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = -INFINITY;
+        if (i < nv && e < E) v[i] = lg[e] + s_bias[e];
       }
     }
     // each lane keeps its best untaken (value, id); only the lane that owned
@@ -218,11 +345,27 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
         }
       }
     };
+    int my_id = -1;
+    float my_v = -INFINITY;
+    if (k <= 8) {
+      float tv[8];
+      int ti[8];
+      warp_top8(lg, s_bias, E, lane, tv, ti);
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r == lane && r < k) {
+          my_id = ti[r];
+          my_v = tv[r];
+        }
+      }
+      if (lane < k && (my_id < 0 || my_id >= E)) {  // cannot happen for k <= E; keep the plan valid
+        atomicCAS(a.status, kStatusOk, kStatusPlan);
+        my_id = lane;
+      }
+    } else {
     float lbv;
     int lbi;
     local_best(lbv, lbi);
-    int my_id = -1;
-    float my_v = -INFINITY;
     for (int j = 0; j < k; ++j) {
       float bv = lbv;
       int bi = lbi;
@@ -240,6 +383,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
         local_best(lbv, lbi);
       }
     }
+    }
     // renormalised weights: p_j / sum_S p = exp(l_j - l_max) / sum_S exp(l_i - l_max)
     const float lmax = __shfl_sync(0xffffffffu, my_v, 0);
     const float ex = (lane < k) ? expf(my_v - lmax) : 0.f;
@@ -253,6 +397,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
       s_ids[t * k + lane] = my_id;
       s_w[t * k + lane] = wj;
     }
+  }
+    __syncthreads();  // the staging buffer is reused by the next group of tokens
   }
   for (int e = tid; e < E; e += kRouterThreads) s_cnt[e] = 0;
   __syncthreads();
@@ -295,18 +441,30 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   }
 
   __syncthreads();
-  // Assignment (t, j) goes to offset[e] + #{t' < t : e in ids[t']} (ids of one
-  // token are distinct, so this orders each expert's assignments by token).
-  for (int i = tid; i < nas; i += kRouterThreads) {
-    const int t = i / k, e = s_ids[i];
-    int rank = 0;
-    for (int i2 = 0; i2 < t * k; ++i2) rank += (s_ids[i2] == e);
-    const int pos = s_off[e] + rank;
-    a.plan->assign_tok[pos] = t;
-    a.plan->assign_slot[pos] = i;
-    a.plan->assign_w[pos] = s_w[i];
+  // Assignment (t, j) goes to offset[e] + #{t' < t : e in ids[t']}: one warp
+  // walks the tokens in order, lane j placing slot j, with a per-expert fill
+  // counter (the ids of one token are distinct, so no two lanes of a step
+  // share a counter); each expert's assignments end up ordered by token.
+  for (int e = tid; e < E; e += kRouterThreads) s_cnt[e] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    for (int t = 0; t < B; ++t) {
+      if (lane < k) {
+        const int i = t * k + lane, e = s_ids[i];
+        const int pos = s_off[e] + s_cnt[e];
+        s_cnt[e] = s_cnt[e] + 1;
+        if (pos < nas) {
+          a.plan->assign_slot[pos] = i;
+          a.plan->assign_w[pos] = s_w[i];
+        }
+      }
+      __syncwarp();
+    }
   }
-  if (tid == 0) *a.ticket = 0u;
+  if (tid == 0) {
+    *a.ticket = 0u;
+    if (a.logits_stride > 0) *a.epoch = *a.epoch + 1u;  // every CTA read it before taking its ticket
+  }
 }
 
 }  // namespace moe

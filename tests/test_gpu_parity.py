@@ -14,6 +14,7 @@ import pytest
 import torch
 
 from moe_decode_block_b200 import MOE_OK, MoEDecode, synth
+import oracle
 from gpu_helpers import Run, margin_x, oracle_check
 
 pytestmark = pytest.mark.gpu
@@ -260,3 +261,32 @@ def test_full_size_two_stream_plan(full, B):
         assert run.blk.status() == MOE_OK
     finally:
         run.blk.close()
+
+
+@pytest.mark.parametrize("plan", PLANS)
+def test_exact_logit_ties_go_to_the_smaller_id(plan):
+    # router columns 2p and 2p+1 identical: their logits are equal in fp64 and
+    # bitwise equal on the GPU (one thread sums both columns in the same order
+    # and one vector reduction adds them), so every selected pair must come
+    # out smaller id first; x is drawn so that distinct pairs keep a margin
+    s = synth.TINY
+    wts = synth.make_weights(s, seed=21, device="cuda")
+    rw = wts.router_w.clone()
+    rw[:, 1::2] = rw[:, 0::2]
+    tied = synth.BlockWeights(rw, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, None)
+    run = Run(s, tied, max_batch=8, two_stream=plan == "two_stream")
+    B = 6
+    rows = []
+    attempt = 0
+    while len(rows) < B:
+        x1 = synth.make_x(1, s.hidden, seed=500 + attempt)
+        attempt += 1
+        logits, _, _ = oracle.router(synth.bf16_bits(x1), synth.bf16_bits(rw), s.top_k, None)
+        pair = np.sort(logits[0, 0::2])[::-1]
+        if pair[0] - pair[1] >= 1e-3:
+            rows.append(x1)
+    x = torch.cat(rows).to("cuda")
+    out, ids, w = run.forward(x)
+    ids_h = ids.cpu().numpy()
+    assert np.all(ids_h[:, 0] % 2 == 0) and np.all(ids_h[:, 1] == ids_h[:, 0] + 1)
+    oracle_check(tied, s.top_k, x, out, ids, w)
