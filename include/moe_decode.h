@@ -81,10 +81,22 @@ extern "C" {
  * router_bias (optional) is a device float32 [n_experts] added to the router
  * logits before softmax and selection; NULL means no bias.  It is read by
  * every forward (the pointer is kept, the data is not copied).
- * flags: 0 or MOE_FLAG_TWO_STREAM (see the top of this file); other bits
- * are rejected with MOE_ERR_UNSUPPORTED_SHAPE.
+ * flags: any combination of MOE_FLAG_TWO_STREAM (see the top of this file)
+ * and MOE_FLAG_TCGEN05 (below); other bits are rejected with
+ * MOE_ERR_UNSUPPORTED_SHAPE.
  */
 #define MOE_FLAG_TWO_STREAM 1u
+/*
+ * MOE_FLAG_TCGEN05: run the expert kernel on the 5th-generation tensor cores
+ * (tcgen05.mma, accumulators in tensor memory, one issuing thread, four
+ * epilogue warps) instead of mma.sync with register accumulators.  Used only
+ * when hidden, inter and shared_inter are multiples of 64 (otherwise the flag
+ * is ignored).  Same results within rounding.  Measured slower on B200 for
+ * 1-64 tokens: with the tokens as the N dimension each tcgen05.mma covers
+ * 128 x 16 weights, so a 64 KB weight stage takes 16 of them, and issuing
+ * those from one thread takes about as long as HBM takes to deliver the stage.
+ */
+#define MOE_FLAG_TCGEN05 2u
 typedef struct moe_decode_shapes {
   int32_t hidden;
   int32_t n_experts;

@@ -36,6 +36,7 @@ EXPORTED = (
 )
 MOE_TIMING_EVENTS = 6
 MOE_FLAG_TWO_STREAM = 1
+MOE_FLAG_TCGEN05 = 2
 
 
 class Shapes(ctypes.Structure):
@@ -145,18 +146,21 @@ def router_topk_noalloc(x, router_w, topk_ids, topk_w, top_k: int, router_bias=N
 class MoEDecode:
     """One MoE block shape bound to the current CUDA device (owns a workspace).
 
-    two_stream=False (default): router kernel + one expert kernel (shared
-    expert, routed experts, combine) on the main stream.  two_stream=True:
-    MOE_FLAG_TWO_STREAM, the shared expert on the aux stream and a separate
-    combine kernel."""
+    two_stream=False (default): router kernel, one expert kernel (shared
+    and routed experts) and the combine on the main stream.  two_stream=True:
+    MOE_FLAG_TWO_STREAM, the shared expert on the aux stream.  tcgen05=True:
+    MOE_FLAG_TCGEN05, the expert kernel on tcgen05 with TMEM accumulators."""
 
     def __init__(self, hidden: int, n_experts: int, top_k: int, inter: int, shared_inter: int = 0,
-                 n_shared: int = 1, max_batch: int = 64, router_bias=None, two_stream: bool = False):
+                 n_shared: int = 1, max_batch: int = 64, router_bias=None, two_stream: bool = False,
+                 tcgen05: bool = False):
         self._lib = load_library()
         self._bias = router_bias  # keep the device tensor alive
         self.two_stream = bool(two_stream)
+        self.tcgen05 = bool(tcgen05)
+        flags = (MOE_FLAG_TWO_STREAM if two_stream else 0) | (MOE_FLAG_TCGEN05 if tcgen05 else 0)
         self.shapes = Shapes(hidden, n_experts, top_k, inter, shared_inter if n_shared else 0, n_shared,
-                             max_batch, _ptr(router_bias), MOE_FLAG_TWO_STREAM if two_stream else 0)
+                             max_batch, _ptr(router_bias), flags)
         h = ctypes.c_void_p()
         _check(self._lib.moe_decode_init(ctypes.byref(self.shapes), ctypes.byref(h)), "moe_decode_init")
         self._h = h

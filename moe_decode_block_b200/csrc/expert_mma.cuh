@@ -400,49 +400,55 @@ __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], float* ba
   }
 }
 
+// Shared-memory pieces of the expert kernels (ring, headers, flags, plan copy).
+struct SmemView {
+  uint8_t* stages;
+  uint64_t* full;
+  uint64_t* empty;
+  StageHdr* hdr;
+  volatile int* s_misc;  // [0]: abort flag (a bounded wait gave up), [2]: stages issued
+  uint16_t* s_uexp;      // [kMaxUnits]
+  uint16_t* s_ubeg;      // [kMaxUnits]
+  uint16_t* s_aslot;     // [kMaxAssign]
+  uint8_t* s_ucnt;       // [kMaxUnits]
+  uint32_t* s_ready;     // [kMaxUnits + kMaxSharedUnits]
+};
+
+// Carve the view out of dynamic shared memory (ring on a 1 KB boundary).
+__device__ __forceinline__ SmemView carve_smem(uint8_t* raw, int NS) {
+  SmemView v;
+  v.stages = raw + ((1024u - (smem_addr(raw) & 1023u)) & 1023u);
+  v.full = reinterpret_cast<uint64_t*>(v.stages + (size_t)NS * kStageBytesMma);
+  v.empty = v.full + kMaxStagesMma;
+  v.hdr = reinterpret_cast<StageHdr*>(v.empty + kMaxStagesMma);
+  v.s_misc = reinterpret_cast<volatile int*>(v.hdr + kMaxStagesMma);
+  v.s_uexp = reinterpret_cast<uint16_t*>(const_cast<int*>(v.s_misc) + 16);
+  v.s_ubeg = v.s_uexp + kMaxUnits;
+  v.s_aslot = v.s_ubeg + kMaxUnits;
+  v.s_ucnt = reinterpret_cast<uint8_t*>(v.s_aslot + kMaxAssign);
+  v.s_ready = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(v.s_uexp) +
+                                          (kMaxUnits * (2 + 2 + 1) + kMaxAssign * 2 + 3) / 4 * 4);
+  return v;
+}
+
+// The producer warp: takes tickets, walks the work list and fills the stage
+// ring (weights by TMA, the stage's token activations, the stage header);
+// ends by posting a kKindEnd header.  Shared by both expert kernels.
 template <int KC, bool TMAP>
-__global__ void __launch_bounds__(expert_threads(KC), 1)
-    expert_mlp_kernel(const __grid_constant__ MmaArgs args, const __grid_constant__ ExpertTable tab13,
-                      const __grid_constant__ ExpertTable tab2) {
-  extern __shared__ __align__(1024) uint8_t mma_smem[];
-  const int NS = args.n_stages;
-  // the ring starts on a 1024-byte boundary (128-byte swizzle atoms)
-  uint8_t* stages = mma_smem + ((1024u - (smem_addr(mma_smem) & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(stages + (size_t)NS * kStageBytesMma);
-  uint64_t* empty = full + kMaxStagesMma;
-  StageHdr* hdr = reinterpret_cast<StageHdr*>(empty + kMaxStagesMma);
-  volatile int* s_misc = reinterpret_cast<volatile int*>(hdr + kMaxStagesMma);
-  // s_misc[0]: abort flag (a bounded wait gave up), [2]: stages issued
-  uint16_t* s_uexp = reinterpret_cast<uint16_t*>(const_cast<int*>(s_misc) + 16);  // [kMaxUnits]
-  uint16_t* s_ubeg = s_uexp + kMaxUnits;                                          // [kMaxUnits]
-  uint16_t* s_aslot = s_ubeg + kMaxUnits;                                         // [kMaxAssign]
-  uint8_t* s_ucnt = reinterpret_cast<uint8_t*>(s_aslot + kMaxAssign);             // [kMaxUnits]
-  uint32_t* s_ready = reinterpret_cast<uint32_t*>(                                // [kMaxUnits + shared]
-      reinterpret_cast<uint8_t*>(s_uexp) + (kMaxUnits * (2 + 2 + 1) + kMaxAssign * 2 + 3) / 4 * 4);
-
-  constexpr int CW = consumer_warps_for(KC);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool is_producer = (warp == CW);
-
-  if (tid == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], CW);
-    }
-    s_misc[0] = 0;
-    s_misc[2] = 0;
-    mbar_fence_init();
-  }
-  __syncthreads();
-
-  const int H = args.H;
+__device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertTable& tab13, const ExpertTable& tab2,
+                                              const SmemView& sv, int NS, unsigned ready_mark, int lane) {
+  uint8_t* stages = sv.stages;
+  uint64_t* full = sv.full;
+  uint64_t* empty = sv.empty;
+  StageHdr* hdr = sv.hdr;
+  volatile int* s_misc = sv.s_misc;
   volatile int* abort_flag = s_misc;
-  // Launch epoch: advanced by the last CTA of the previous launch on this
-  // workspace, which finished before the previous grid (the router) passed
-  // its own dependency wait; every CTA of this launch reads the same value.
-  const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
-
-  if (is_producer) {
+  uint16_t* s_uexp = sv.s_uexp;
+  uint16_t* s_ubeg = sv.s_ubeg;
+  uint16_t* s_aslot = sv.s_aslot;
+  uint8_t* s_ucnt = sv.s_ucnt;
+  uint32_t* s_ready = sv.s_ready;
+  const int H = args.H;
     // ================================================================ producer
     const uint64_t pol = l2_evict_first_policy();
     const int G = gridDim.x;
@@ -732,6 +738,45 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       hdr[slot].kind = kKindEnd;
       mbar_arrive(&full[slot]);
     }
+}
+
+template <int KC, bool TMAP>
+__global__ void __launch_bounds__(expert_threads(KC), 1)
+    expert_mlp_kernel(const __grid_constant__ MmaArgs args, const __grid_constant__ ExpertTable tab13,
+                      const __grid_constant__ ExpertTable tab2) {
+  extern __shared__ __align__(1024) uint8_t mma_smem[];
+  const int NS = args.n_stages;
+  const SmemView sv = carve_smem(mma_smem, NS);
+  uint8_t* stages = sv.stages;
+  uint64_t* full = sv.full;
+  uint64_t* empty = sv.empty;
+  StageHdr* hdr = sv.hdr;
+  volatile int* s_misc = sv.s_misc;
+
+  constexpr int CW = consumer_warps_for(KC);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool is_producer = (warp == CW);
+
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], CW);
+    }
+    s_misc[0] = 0;
+    s_misc[2] = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  const int H = args.H;
+  volatile int* abort_flag = s_misc;
+  // Launch epoch: advanced by the last CTA of the previous launch on this
+  // workspace, which finished before the previous grid (the router) passed
+  // its own dependency wait; every CTA of this launch reads the same value.
+  const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
+
+  if (is_producer) {
+    producer_loop<KC, TMAP>(args, tab13, tab2, sv, NS, ready_mark, lane);
   } else {
     // =============================================================== consumers
     // (they read nothing the router writes: the stage headers carry it)

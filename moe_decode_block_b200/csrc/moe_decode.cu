@@ -30,6 +30,7 @@
 #include "moe_decode.h"
 #include "combine.cuh"
 #include "expert_mma.cuh"
+#include "expert_tc.cuh"
 #include "moe_device.cuh"
 #include "router_topk.cuh"
 
@@ -60,7 +61,7 @@ bool shapes_valid(const moe_decode_shapes* s) {
   if (s->n_shared != 0 && s->n_shared != 1) return false;
   if (s->n_shared == 1 && (!in(s->shared_inter, 8, 16384) || s->shared_inter % 8)) return false;
   if (!in(s->max_batch, 1, moe::kMaxBatch)) return false;
-  if ((s->flags & ~MOE_FLAG_TWO_STREAM) != 0) return false;
+  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05)) != 0) return false;
   return true;
 }
 
@@ -225,6 +226,7 @@ struct moe_decode_ctx {
   ExpertTable* tab_none = nullptr;  // zero table passed to the shared-expert launch
   // tensor-map path: maps encoded for the pointer tables of the last forward
   bool use_tmap = false;
+  bool use_tc = false;  // tcgen05 expert kernel (tensor-map path only)
   uint8_t* maps_host = nullptr;  // pinned staging, (2E + 2) maps
   std::vector<const void*> map_ptrs;  // w13[E], w2[E], shared w13, shared w2 the maps describe
   bool maps_uploaded = false;
@@ -281,6 +283,9 @@ int set_kernel_attrs(const moe_decode_ctx* h) {
       if (e != cudaSuccess) return fail_cuda(e);
     }
   }
+  e = cudaFuncSetAttribute(moe::expert_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)moe::tc_smem_bytes(h->n_stages));
+  if (e != cudaSuccess) return fail_cuda(e);
   const int rsmem = (int)moe::router_smem_bytes(h->s.max_batch, h->s.n_experts, h->router_chunk_rows);
   e = cudaFuncSetAttribute(pick_router(h->s.n_experts), cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
   if (e != cudaSuccess) return fail_cuda(e);
@@ -347,11 +352,11 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   int* status = h->at<int>(h->L.status);
   const bool two_stream = (s.flags & MOE_FLAG_TWO_STREAM) != 0;
   const bool fork = two_stream && s.n_shared && sa != sm;
-  const size_t smem = moe::mma_smem_bytes(h->n_stages);
   const int n_su = shared_units(s, batch);
   const int kc = kernel_class(batch);
-  const MlpKernel mlp = pick_mlp(kc, h->use_tmap);
-  const int mlp_threads = moe::expert_threads(kc);
+  const MlpKernel mlp = h->use_tc ? moe::expert_tc_kernel : pick_mlp(kc, h->use_tmap);
+  const int mlp_threads = h->use_tc ? moe::kTcThreads : moe::expert_threads(kc);
+  const size_t smem = h->use_tc ? moe::tc_smem_bytes(h->n_stages) : moe::mma_smem_bytes(h->n_stages);
 
   auto bail = [&](cudaError_t err) {
     h->dirty = true;
@@ -733,6 +738,7 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
     uint8_t probe[moe::kTensorMapBytes];
     h->use_tmap = env_int("MOE_DECODE_TMAP", 1, 0, 1) == 1 && shapes_ok &&
                   encode_matrix_map(probe, h->ws, shapes->hidden, 2 * shapes->inter);
+    h->use_tc = h->use_tmap && (shapes->flags & MOE_FLAG_TCGEN05) != 0;
     if (h->use_tmap) {
       h->map_ptrs.assign(2 * (size_t)shapes->n_experts + 2, nullptr);
       e = cudaMallocHost(reinterpret_cast<void**>(&h->maps_host),

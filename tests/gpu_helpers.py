@@ -39,12 +39,12 @@ def margin_x(batch, hidden, wts, k, seed=0, device="cuda", min_gap=MIN_MARGIN):
 class Run:
     """Device buffers and one handle for a block shape."""
 
-    def __init__(self, shape: synth.BlockShape, wts, max_batch=64, two_stream=False):
+    def __init__(self, shape: synth.BlockShape, wts, max_batch=64, two_stream=False, tcgen05=False):
         self.s = shape
         self.wts = wts
         self.blk = MoEDecode(shape.hidden, shape.n_experts, shape.top_k, shape.inter, shape.shared_inter,
                              n_shared=shape.n_shared, max_batch=max_batch, router_bias=wts.router_bias,
-                             two_stream=two_stream)
+                             two_stream=two_stream, tcgen05=tcgen05)
 
     def kernels_per_forward(self):
         """Kernels one forward enqueues: router, expert kernel, combine by default;

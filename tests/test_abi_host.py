@@ -65,7 +65,7 @@ def test_workspace_bytes_and_shape_validation(lib):
     assert 0 < tiny < full
     bad = [dict(hidden=7170), dict(hidden=0), dict(n_experts=12), dict(n_experts=2048), dict(top_k=0),
            dict(top_k=33), dict(top_k=9, n_experts=8), dict(inter=100), dict(n_shared=2),
-           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=2), dict(flags=3)]
+           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=4), dict(flags=5)]
     for kw in bad:
         sh = _shapes(**kw)
         assert lib.moe_decode_workspace_bytes(ctypes.byref(sh)) == 0, kw
@@ -74,6 +74,8 @@ def test_workspace_bytes_and_shape_validation(lib):
         assert not h.value
     # the two-stream plan flag is accepted and needs the same workspace
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TWO_STREAM))) == full
+    assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TCGEN05))) == full
+    assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=3))) == full
     # shared_inter is ignored when there is no shared expert
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(n_shared=0, shared_inter=0))) > 0
 

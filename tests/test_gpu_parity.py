@@ -23,10 +23,11 @@ pytestmark = pytest.mark.gpu
 PLANS = ["default", "two_stream"]
 
 
-@pytest.fixture(scope="module", params=PLANS)
+@pytest.fixture(scope="module", params=PLANS + ["tcgen05"])
 def tiny(request):
     wts = synth.make_weights(synth.TINY, seed=0, device="cuda")
-    return Run(synth.TINY, wts, max_batch=64, two_stream=request.param == "two_stream")
+    return Run(synth.TINY, wts, max_batch=64, two_stream=request.param == "two_stream",
+               tcgen05=request.param == "tcgen05")
 
 
 @pytest.fixture(scope="module")
@@ -247,6 +248,20 @@ def test_graph_replay_alternating_inputs_full_b8(full):
     xa = margin_x(8, synth.FULL.hidden, full.wts, 8, seed=11)
     xb = margin_x(8, synth.FULL.hidden, full.wts, 8, seed=12)
     _graph_alternating(full, xa, xb, replays=5)
+
+
+@pytest.mark.parametrize("B", [1, 8, 40])
+def test_full_size_tcgen05_expert_kernel(full, B):
+    # the expert kernel on tcgen05 with TMEM accumulators (MOE_FLAG_TCGEN05)
+    run = Run(synth.FULL, full.wts, max_batch=64, tcgen05=True)
+    try:
+        x = margin_x(B, synth.FULL.hidden, full.wts, synth.FULL.top_k, seed=300 + B)
+        out, ids, w = run.forward(x)
+        rows = np.unique(np.linspace(0, B - 1, min(B, 4)).astype(int))
+        oracle_check(full.wts, synth.FULL.top_k, x, out, ids, w, rows=rows)
+        assert run.blk.status() == MOE_OK
+    finally:
+        run.blk.close()
 
 
 @pytest.mark.parametrize("B", [1, 8, 40])
