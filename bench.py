@@ -192,9 +192,10 @@ def host_oracle_inputs(wl, wts, x, ids_np):
                 sw13=synth.bf16_bits(wts.shared_w13), sw2=synth.bf16_bits(wts.shared_w2), bias=bias)
 
 
-def time_oracle(wl, inp, bytes_step, min_seconds=10.0, max_runs=30, warmup=1, max_seconds=None):
+def time_oracle(wl, inp, bytes_step, min_seconds=10.0, max_runs=30, warmup=1, max_seconds=None, warmup_seconds=None):
     """The fp64 oracle, as it stands, on the host cores: router + block for
-    the whole batch per run.  Returns (GB/s, seconds per run, runs, threads)."""
+    the whole batch per run.  Returns (GB/s, seconds per run, runs, threads,
+    warm-up runs done); warm-up stops early after warmup_seconds."""
     import oracle
     k = wl.shape.top_k
 
@@ -202,8 +203,13 @@ def time_oracle(wl, inp, bytes_step, min_seconds=10.0, max_runs=30, warmup=1, ma
         _, ids, w = oracle.router(inp["x"], inp["R"], k, inp["bias"])
         oracle.block(inp["x"], ids, w, inp["h13"], inp["h2"], inp["sw13"], inp["sw2"], n_experts=wl.shape.n_experts)
 
+    done_warmup = 0
+    t_w = time.perf_counter()
     for _ in range(warmup):
         one()
+        done_warmup += 1
+        if warmup_seconds is not None and time.perf_counter() - t_w >= warmup_seconds:
+            break
     times = []
     t_start = time.perf_counter()
     while len(times) < max_runs:
@@ -216,7 +222,7 @@ def time_oracle(wl, inp, bytes_step, min_seconds=10.0, max_runs=30, warmup=1, ma
         if max_seconds is not None and el >= max_seconds:
             break
     per = statistics.median(times)
-    return bytes_step / per / 1e9, per, len(times), oracle.num_threads()
+    return bytes_step / per / 1e9, per, len(times), oracle.num_threads(), done_warmup
 
 
 # -------------------------------------------------------------------- arms --
@@ -242,11 +248,12 @@ def run_reference(args):
     bstep, distinct = bytes_per_step(wl.shape, ids, wl.batch)
     inp = host_oracle_inputs(wl, wts, x, ids)
     budget = 120.0
-    gbs, per, runs, threads = time_oracle(wl, inp, bstep, min_seconds=float("inf"), max_runs=max(1, args.steps),
-                                          warmup=min(args.warmup, 1), max_seconds=budget)
+    gbs, per, runs, threads, warm = time_oracle(wl, inp, bstep, min_seconds=float("inf"),
+                                                max_runs=max(1, args.steps), warmup=args.warmup,
+                                                max_seconds=budget, warmup_seconds=30.0)
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": args.gpus,
-        "steps": runs, "steps_requested": args.steps, "warmup": min(args.warmup, 1),
+        "steps": runs, "steps_requested": args.steps, "warmup": warm, "warmup_requested": args.warmup,
         "ms_per_step": round(per * 1e3, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
         "config": _config_dict(wl, graph=False),
@@ -443,7 +450,7 @@ def run_ours(args):
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         inp = host_oracle_inputs(wl, wts, x, ids.cpu().numpy())
-        gbs, per, runs, threads = time_oracle(wl, inp, bstep, min_seconds=10.0, max_runs=30)
+        gbs, per, runs, threads, _ = time_oracle(wl, inp, bstep, min_seconds=10.0, max_runs=30)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{runs} full forwards of the {wl.name} block (router + {distinct} routed + shared "
                          f"expert MLPs) by the fp64 C oracle, >= 10 s of CPU work, median "
