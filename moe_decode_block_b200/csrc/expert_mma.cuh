@@ -87,28 +87,33 @@ namespace moe {
 
 constexpr int kUnitTok = kMaxUnitTokens;  // tokens of one unit, at most
 constexpr int kNumClasses = 3;
-__host__ __device__ constexpr int class_lw(int c) { return c <= 1 ? 2048 : 1024; }
-__host__ __device__ constexpr int class_rows(int c) { return c <= 1 ? 16 : 32; }
+// Token classes.  A unit with more tokens takes a narrower panel of more
+// rows, so every stage holds lw x rows = 32K weights (64 KB) and every
+// consumer warp keeps the same eight accumulator fragments (32 floats) in
+// every class: 2048 x 16 for 1-8 tokens (one 8-token tile), 1024 x 32 for
+// 9-16 (two tiles), 512 x 64 for 17-32 (four tiles).
+__host__ __device__ constexpr int class_lw(int c) { return c == 0 ? 2048 : (c == 1 ? 1024 : 512); }
+__host__ __device__ constexpr int class_rows(int c) { return c == 0 ? 16 : (c == 1 ? 32 : 64); }
 __host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : 4); }
 // class of a unit with n <= kUnitTok tokens
 __host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : 2); }
-// Consumer warps of the instance compiled for classes <= kc: sixteen when a
-// thread needs only 32 accumulators (more warps hide more latency), eight
-// otherwise -- nine warps per CTA leave each thread 168 registers, enough for
-// 128 accumulators, where seventeen warps cap it at 96.
-__host__ __device__ constexpr int consumer_warps_for(int kc) { return kc == 0 ? 16 : 8; }
+// Consumer warps: sixteen in every instance (seventeen warps with the
+// producer cap a thread at 96 registers, room for the 32 accumulators).
+__host__ __device__ constexpr int consumer_warps_for(int) { return 16; }
 __host__ __device__ constexpr int expert_threads(int kc) { return (consumer_warps_for(kc) + 1) * 32; }
 // m-tiles (16 columns) per consumer warp for class c with cw consumer warps
 __host__ __device__ constexpr int class_mt(int c, int cw) { return class_lw(c) / (cw * 16); }
 // accumulator fragments (of 4 floats) a consumer thread needs for classes <= KC
-__host__ __device__ constexpr int acc_frags(int kc) {
-  return kc == 0 ? class_mt(0, consumer_warps_for(0)) * class_nt(0)
-                 : class_mt(1, consumer_warps_for(kc)) * class_nt(1);
-}
-static_assert(class_mt(2, 8) * class_nt(2) == acc_frags(2), "class 2 fits the class 1 budget");
-constexpr int kStageWBytes = 65536 + 32 * 16;                // rows * (2*LW + 16), largest over classes
-constexpr int kStageXBytes = kUnitTok * (32 * 2 + 16);       // tokens * (2*rows + 16), largest
-constexpr int kStageBytesMma = kStageWBytes + kStageXBytes;  // 68608 = 67 KB (stages stay 1 KB aligned)
+__host__ __device__ constexpr int acc_frags(int kc) { return class_mt(0, consumer_warps_for(kc)) * class_nt(0); }
+static_assert(class_mt(1, 16) * class_nt(1) == acc_frags(1) && class_mt(2, 16) * class_nt(2) == acc_frags(2),
+              "every class keeps the same accumulators");
+// stage buffers: weights (row pitch 2*lw + 16 on the plain-copy path) and
+// the tokens' activation rows (pitch 2*rows + 16), largest over the classes
+__host__ __device__ constexpr int stage_w_bytes(int c) { return class_rows(c) * (class_lw(c) * 2 + 16); }
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
+constexpr int kStageWBytes = cmax(stage_w_bytes(0), cmax(stage_w_bytes(1), stage_w_bytes(2)));  // 66560
+constexpr int kStageXBytes = kUnitTok * (class_rows(2) * 2 + 16);                                 // 4608
+constexpr int kStageBytesMma = (kStageWBytes + kStageXBytes + 1023) / 1024 * 1024;               // 70 KB
 static_assert(kStageBytesMma % 1024 == 0, "128-byte swizzle atoms need 1 KB aligned stages");
 constexpr int kMaxStagesMma = 3;
 constexpr int kMaxChunk = 64;  // stages per queue grab, at most
@@ -119,7 +124,7 @@ constexpr int kBoxChunks = 4;
 constexpr int kChunkTile = kBoxRows * kChunkCols * 2;  // 2048 B: one chunk of one 16-row block
 constexpr int kBoxBytes = kChunkTile * kBoxChunks;     // 8192 B per load
 constexpr int kTensorMapBytes = 128;
-// UP panels of a unit, at most: ceil(I / 512) (class 2); sizes the panel counters
+// UP panels of a unit, at most: ceil(I / 256) (class 2); sizes the panel counters
 __host__ __device__ inline int max_up_panels(int I) { return (I + class_lw(2) / 2 - 1) / (class_lw(2) / 2); }
 
 enum : int { kKindUp = 0, kKindDown = 1, kKindEnd = 2 };
@@ -296,8 +301,9 @@ __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint
     const int k0 = ks * 16;
     if (k0 >= nrows) break;
     const bool half = (nrows - k0) < 16;  // only 8 valid rows in this k-step
-    // token fragments: kept for all tiles when there are few of them, loaded
-    // per m-tile otherwise (keeps the accumulators in registers)
+    // token fragments: loaded once per k-step and kept for all m-tiles with
+    // up to two tiles; four tiles (class 2) are reloaded per m-tile, which
+    // measured faster than keeping them (that costs a spill)
     constexpr bool kKeepB = NT <= 2;
     uint32_t b[kKeepB ? NT : 1][2];
     auto load_b = [&](int nt, uint32_t& b0, uint32_t& b1) {
@@ -630,8 +636,9 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         if (!up) {
           const int need_p = row0 / (lw / 2);
           const int need_panel = unit * (seg == 0 ? args.panel_stride_s : args.panel_stride) + need_p;
+          // (panels past the 32 this CTA caches a bit for are polled each time)
           uint32_t* seen = s_ready + (seg == 0 ? kMaxUnits + unit : unit);
-          if (!((*seen >> need_p) & 1u)) {
+          if (need_p >= 32 || !((*seen >> need_p) & 1u)) {
             const unsigned* pr = (seg == 0 ? args.panel_ready_s : args.panel_ready) + need_panel;
             int ok = 1;
             if (lane == 0) {
@@ -654,7 +661,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
               stop = true;
               break;
             }
-            if (lane == 0) *seen |= 1u << need_p;
+            if (lane == 0 && need_p < 32) *seen |= 1u << need_p;
             __syncwarp();
           }
         }

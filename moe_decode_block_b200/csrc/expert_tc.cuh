@@ -29,7 +29,7 @@ namespace moe {
 constexpr int kTcThreads = 6 * 32;      // producer, MMA, 4 epilogue warps
 constexpr int kTmemCols = 512;          // two accumulator buffers of 256 columns
 constexpr int kTmemBufCols = 256;
-constexpr int kTcBBytes = kUnitTok * 32 * 2;  // B operand: 32 tokens x 32 rows bf16 (largest class)
+constexpr int kTcBBytes = kUnitTok * class_rows(2) * 2;  // B operand: 32 tokens x 64 rows bf16 (largest class)
 
 // Shared memory of expert_tc_kernel: the expert_mlp_kernel layout, then the
 // B-operand buffers, two piece descriptors, the accumulator barriers and the

@@ -210,7 +210,8 @@ struct moe_decode_ctx {
   moe_decode_shapes s{};
   int device = 0;
   int num_sms = 0;
-  int n_stages = 3;
+  int n_stages = 3;     // stage ring depth of expert_mlp_kernel
+  int n_stages_tc = 2;  // of expert_tc_kernel (its B-operand buffers take room)
   int grid_routed = 0, grid_shared = 0, grid_router_max = 0;
   bool grid_routed_auto = true;
   int router_chunk_rows = 0;
@@ -284,7 +285,7 @@ int set_kernel_attrs(const moe_decode_ctx* h) {
     }
   }
   e = cudaFuncSetAttribute(moe::expert_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)moe::tc_smem_bytes(h->n_stages));
+                           (int)moe::tc_smem_bytes(h->n_stages_tc));
   if (e != cudaSuccess) return fail_cuda(e);
   const int rsmem = (int)moe::router_smem_bytes(h->s.max_batch, h->s.n_experts, h->router_chunk_rows);
   e = cudaFuncSetAttribute(pick_router(h->s.n_experts), cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
@@ -356,7 +357,8 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   const int kc = kernel_class(batch);
   const MlpKernel mlp = h->use_tc ? moe::expert_tc_kernel : pick_mlp(kc, h->use_tmap);
   const int mlp_threads = h->use_tc ? moe::kTcThreads : moe::expert_threads(kc);
-  const size_t smem = h->use_tc ? moe::tc_smem_bytes(h->n_stages) : moe::mma_smem_bytes(h->n_stages);
+  const int n_stages = h->use_tc ? h->n_stages_tc : h->n_stages;
+  const size_t smem = h->use_tc ? moe::tc_smem_bytes(n_stages) : moe::mma_smem_bytes(n_stages);
 
   auto bail = [&](cudaError_t err) {
     h->dirty = true;
@@ -373,7 +375,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.Is = s.n_shared ? s.shared_inter : 0;
   base.E = s.n_experts;
   base.top_k = s.top_k;
-  base.n_stages = h->n_stages;
+  base.n_stages = n_stages;
   base.batch = batch;
   base.max_units = (int)max_units(&s);
   base.panel_stride = moe::max_up_panels(s.inter);
@@ -692,6 +694,11 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
   h->n_stages = env_int("MOE_DECODE_STAGES", 3, 2, moe::kMaxStagesMma);
+  // the deepest rings that fit the opt-in shared memory of a block
+  const size_t smem_max = prop.sharedMemPerBlockOptin;
+  while (h->n_stages > 2 && moe::mma_smem_bytes(h->n_stages) > smem_max) --h->n_stages;
+  h->n_stages_tc = h->n_stages;
+  while (h->n_stages_tc > 2 && moe::tc_smem_bytes(h->n_stages_tc) > smem_max) --h->n_stages_tc;
   h->grid_routed = env_int("MOE_DECODE_GRID_ROUTED", 0, 0, 8 * h->num_sms);
   h->grid_routed_auto = h->grid_routed == 0;
   if (h->grid_routed == 0) h->grid_routed = h->num_sms;

@@ -68,10 +68,15 @@ WORKLOADS: Dict[str, Workload] = {
     "full_b64": Workload("full_b64", FULL, 64, "uniform", "full-size block, batch 64, uniform-ish routing"),
     "zipf_b32": Workload("zipf_b32", FULL, 32, "zipf",
                          "full-size block, batch 32, Zipf(1.2) per-expert log-prior added to router logits"),
+    **{f"zipf_b{b}": Workload(f"zipf_b{b}", FULL, b, "zipf",
+                              f"full-size block, batch {b}, Zipf(1.2) log-prior (batch sweep)")
+       for b in (1, 2, 4, 8, 16, 64)},
     "prof_b1": Workload("prof_b1", PROF, 1, "uniform",
                         "profiling case: full-size experts, 16 of them (1.4 GB), batch 1"),
     "prof_b8": Workload("prof_b8", PROF, 8, "uniform",
                         "profiling case: full-size experts, 16 of them (1.4 GB), batch 8"),
+    "prof_b64": Workload("prof_b64", PROF, 64, "uniform",
+                         "profiling case: full-size experts, 16 of them (1.4 GB), batch 64 (~32 tokens per expert)"),
 }
 
 
