@@ -444,7 +444,8 @@ def run_ours(args):
             e2e_val = bstep * world / float(t.item()) / 1e9
         e2e = {"value": round(e2e_val, 2), "unit": "GB/s", "us_per_block": round(e2e_s * 1e6, 1),
                "h2d_bytes_per_step": B * s.hidden * 2, "d2h_bytes_per_step": B * s.hidden * 2 + B * s.top_k * 8,
-               "api": "moe_decode_forward_host (pinned host x in; out, topk_ids, topk_w back; synchronous)"}
+               "api": "moe_decode_forward_host (pinned host buffers: x copied in; out, topk_ids, topk_w "
+                      "stored into them by the kernels; synchronous)"}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N == 1)
     cpu = None

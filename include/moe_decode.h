@@ -177,9 +177,14 @@ int moe_decode_forward(moe_decode_t h, const void* x, const void* router_w,
 /*
  * Same computation with the per-step tensors in HOST memory: copies x_host
  * (bf16 [batch, hidden]) to the handle's device staging buffer, runs the
- * forward, copies out/topk_ids/topk_w back to out_host/ids_host/w_host and
+ * forward, delivers out/topk_ids/topk_w to out_host/ids_host/w_host and
  * synchronises stream_main before returning.  Weights stay device pointers.
- * Pinned host buffers give the fastest copies; pageable ones work.
+ * When out_host (16-byte aligned), ids_host and w_host are all pinned host
+ * memory mapped into the device's address space (cudaHostAlloc'ed or
+ * registered memory on a unified-addressing system), the kernels store the
+ * results into them directly; otherwise the results go through device
+ * staging buffers and three device-to-host copies.  Pinned buffers give the
+ * fastest transfers; pageable ones work.
  */
 int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* router_w,
                             const void* const* w13, const void* const* w2,

@@ -204,6 +204,20 @@ bool encode_matrix_map(uint8_t* out, const void* base, int rows, int cols) {
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// Address at which the current device can write the host buffer `p` (pinned
+// host memory mapped into the device's address space), or nullptr when it
+// has none (pageable memory) or is not aligned to `align` bytes.  Asked anew
+// on every call: a buffer can be unpinned and its address reused.
+void* host_buffer_device_view(void* p, uintptr_t align) {
+  if ((reinterpret_cast<uintptr_t>(p) & (align - 1)) != 0) return nullptr;
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 }  // namespace
 
 struct moe_decode_ctx {
@@ -252,6 +266,10 @@ RouterKernel pick_router(int n_experts) {
   if (n_experts <= 256) return moe::router_topk_kernel<8>;
   if (n_experts <= 512) return moe::router_topk_kernel<16>;
   return moe::router_topk_kernel<32>;
+}
+// Threads of the router kernel pick_router returns.
+int router_threads_for(int n_experts) {
+  return moe::router_threads(n_experts <= 128 ? 4 : (n_experts <= 256 ? 8 : (n_experts <= 512 ? 16 : 32)));
 }
 
 // CTAs for the shared expert when it runs beside the routed experts: its
@@ -422,7 +440,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   auto launch_router = [&]() -> cudaError_t {
     cudaError_t err = mark(0, sm);
     if (err != cudaSuccess) return err;
-    err = launch(pick_router(s.n_experts), ra.G, moe::kRouterThreads,
+    err = launch(pick_router(s.n_experts), ra.G, router_threads_for(s.n_experts),
                  moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra);
     if (err != cudaSuccess) return err;
     ++kernels;
@@ -660,7 +678,7 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
     e = cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail_cuda(e);
   }
-  e = launch(rk, ra.G, moe::kRouterThreads, smem, st, false, ra);
+  e = launch(rk, ra.G, router_threads_for(n_experts), smem, st, false, ra);
   if (e != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }
@@ -791,14 +809,25 @@ int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* rout
   void* od = h->at<void>(h->L.out_stage);
   int32_t* idd = h->at<int32_t>(h->L.ids_stage);
   float* wd = h->at<float>(h->L.w_stage);
+  // Outputs: when all three host buffers are pinned and mapped, the router
+  // and the combine kernel store into them directly (their writes cross the
+  // host link as the kernels run; no copies and no copy latencies after the
+  // last kernel); otherwise through device staging and three copies.
+  void* od_m = host_buffer_device_view(out_host, 16);
+  void* idd_m = od_m ? host_buffer_device_view(ids_host, 4) : nullptr;
+  void* wd_m = idd_m ? host_buffer_device_view(w_host, 4) : nullptr;
+  const bool direct = od_m && idd_m && wd_m;
   cudaError_t e;
   if ((e = cudaMemcpyAsync(xd, x_host, xb, cudaMemcpyHostToDevice, sm)) != cudaSuccess) return fail_cuda(e);
-  rc = enqueue_forward(h, xd, router_w, w13, w2, shared_w13, shared_w2, od, idd, wd, batch, sm,
-                       static_cast<cudaStream_t>(stream_aux));
+  rc = enqueue_forward(h, xd, router_w, w13, w2, shared_w13, shared_w2, direct ? od_m : od,
+                       static_cast<int32_t*>(direct ? idd_m : idd), static_cast<float*>(direct ? wd_m : wd), batch,
+                       sm, static_cast<cudaStream_t>(stream_aux));
   if (rc != MOE_OK) return rc;
-  if ((e = cudaMemcpyAsync(out_host, od, xb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);
-  if ((e = cudaMemcpyAsync(ids_host, idd, kb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);
-  if ((e = cudaMemcpyAsync(w_host, wd, kb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);
+  if (!direct) {
+    if ((e = cudaMemcpyAsync(out_host, od, xb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaMemcpyAsync(ids_host, idd, kb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);
+    if ((e = cudaMemcpyAsync(w_host, wd, kb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);
+  }
   if ((e = cudaStreamSynchronize(sm)) != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }

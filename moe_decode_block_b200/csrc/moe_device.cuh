@@ -19,9 +19,6 @@ constexpr int kMaxAssign = kMaxBatch * kMaxTopK;
 constexpr int kMaxUnitTokens = 32;
 constexpr int kMaxUnits = kMaxExperts + kMaxAssign / kMaxUnitTokens;
 
-
-constexpr int kRouterThreads = 256;
-
 // Device status word values (the host maps them to MOE_ERR_*).
 constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;

@@ -12,9 +12,10 @@
 //     is staged in shared memory with TMA bulk copies issued *before* the
 //     grid-dependency wait (router_w is a static weight, so reading it early
 //     under programmatic dependent launch is safe); x is read only after it.
-//   * Each thread owns a pair of expert columns and accumulates the partial
-//     logits of every token over the slab in fp32; partials are reduced into
-//     a global fp32 [B, E] buffer with vector reductions (red, no return).
+//   * A work item is a pair of expert columns and a group of 8 tokens; a
+//     thread accumulates the item's partial logits over the slab in fp32, and
+//     partials are reduced into a global fp32 [B, E] buffer with vector
+//     reductions (red, no return).
 //   * The last CTA to finish (ticket counter) stages the logits in shared
 //     memory (one batched load per group of tokens), adds the optional bias,
 //     selects the top k per token with warp argmax rounds, computes the
@@ -153,7 +154,8 @@ __device__ __forceinline__ void warp_top8(const float* lg, const float* bias, in
   }
 }
 
-// Exclusive scan of one int per thread over the block (kRouterThreads).
+// Exclusive scan of one int per thread over the block (NT threads).
+template <int NT>
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int inc = v;
@@ -165,31 +167,38 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
   if (lane == 31) warp_tot[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int t = lane < kRouterThreads / 32 ? warp_tot[lane] : 0;
+    int t = lane < NT / 32 ? warp_tot[lane] : 0;
     int ti = t;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       int o = __shfl_up_sync(0xffffffffu, ti, off);
       if (lane >= off) ti += o;
     }
-    if (lane < kRouterThreads / 32) warp_tot[lane] = ti - t;  // exclusive warp offsets
-    if (lane == kRouterThreads / 32 - 1) warp_tot[kRouterThreads / 32] = ti;
+    if (lane < NT / 32) warp_tot[lane] = ti - t;  // exclusive warp offsets
+    if (lane == NT / 32 - 1) warp_tot[NT / 32] = ti;
   }
   __syncthreads();
   const int r = warp_tot[warp] + inc - v;
-  total = warp_tot[kRouterThreads / 32];
+  total = warp_tot[NT / 32];
   __syncthreads();
   return r;
 }
 
 // NV: logits per lane a warp holds in registers during top-k (E <= 32 * NV).
+// Threads: 512 up to 512 experts -- sixteen warps share the last CTA's
+// per-token top-k and the GEMV's (expert pair, token group) items -- and 256
+// above, where a lane's 32 logits need more than the 128 registers a
+// 512-thread block leaves.
+__host__ __device__ constexpr int router_threads(int nv) { return nv <= 16 ? 512 : 256; }
+
 template <int NV>
-__global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __grid_constant__ RouterArgs a) {
+__global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(const __grid_constant__ RouterArgs a) {
+  constexpr int NT = router_threads(NV);
   extern __shared__ __align__(1024) uint8_t router_smem[];
   uint8_t* smem = router_smem;
   __shared__ __align__(8) uint64_t bar;
   __shared__ int s_last;
-  __shared__ int s_warp[kRouterThreads / 32 + 1];
+  __shared__ int s_warp[NT / 32 + 1];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E, B = a.B, H = a.H, k = a.k;
@@ -223,7 +232,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
     float4* other = reinterpret_cast<float4*>(a.logits + (size_t)(par ^ 1u) * a.logits_stride);
     const int n4 = a.logits_stride / 4;
     const int c0 = (int)((long long)n4 * blockIdx.x / a.G), c1 = (int)((long long)n4 * (blockIdx.x + 1) / a.G);
-    for (int i = c0 + tid; i < c1; i += kRouterThreads) __stcg(other + i, make_float4(0.f, 0.f, 0.f, 0.f));
+    for (int i = c0 + tid; i < c1; i += NT) __stcg(other + i, make_float4(0.f, 0.f, 0.f, 0.f));
   }
 
   uint32_t phase = 0;
@@ -233,15 +242,19 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
     const int nr = min(a.chunk_rows, h1 - r0);
     // x staged as [row][token] (tokens padded to 8 with zeros), so a row's
     // 8-token group is two 16-byte shared loads
-    for (int i = tid; i < bp * nr; i += kRouterThreads) {
+    for (int i = tid; i < bp * nr; i += NT) {
       const int r = i / bp, t = i - r * bp;
       xs[i] = t < B ? __bfloat162float(a.x[(size_t)t * H + r0 + r]) : 0.f;
     }
     mbar_wait_bounded(&bar, phase, a.status);
     phase ^= 1;
     __syncthreads();
-    for (int p = tid; p < npairs; p += kRouterThreads) {
-      for (int t0 = 0; t0 < B; t0 += 8) {
+    // items: (expert pair, group of 8 tokens); a warp's lanes take
+    // consecutive pairs of one group
+    const int n_items = npairs * ((B + 7) / 8);
+    for (int it = tid; it < n_items; it += NT) {
+      {
+        const int t0 = (it / npairs) * 8, p = it - (it / npairs) * npairs;
         float acc[8][2];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = 0.f;
@@ -290,7 +303,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
 
   float* s_bias = reinterpret_cast<float*>(s_act + E);  // [E] (16-byte aligned: E % 8 == 0)
   float* s_lg = s_bias + E;                                 // [TB, E]
-  for (int e = tid; e < E; e += kRouterThreads) s_bias[e] = a.bias ? a.bias[e] : 0.f;
+  for (int e = tid; e < E; e += NT) s_bias[e] = a.bias ? a.bias[e] : 0.f;
   const int nv = (E + 31) / 32;
   const int TB = router_stage_tokens(B, E);
   for (int tb0 = 0; tb0 < B; tb0 += TB) {
@@ -300,16 +313,16 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
       float4* src = reinterpret_cast<float4*>(lg_buf + (size_t)tb0 * E);
       float4* dst = reinterpret_cast<float4*>(s_lg);
       const int n4 = ntb * E / 4;
-      for (int i0 = 0; i0 < n4; i0 += 8 * kRouterThreads) {
+      for (int i0 = 0; i0 < n4; i0 += 8 * NT) {
         float4 v[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int i = i0 + u * kRouterThreads + tid;
+          const int i = i0 + u * NT + tid;
           if (i < n4) v[u] = __ldcg(src + i);
         }
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int i = i0 + u * kRouterThreads + tid;
+          const int i = i0 + u * NT + tid;
           if (i < n4) {
             dst[i] = v[u];
             if (a.logits_stride == 0) __stcg(src + i, make_float4(0.f, 0.f, 0.f, 0.f));
@@ -318,7 +331,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
       }
     }
     __syncthreads();
-  for (int t = tb0 + warp; t < tb0 + ntb; t += kRouterThreads / 32) {
+  for (int t = tb0 + warp; t < tb0 + ntb; t += NT / 32) {
     const float* lg = s_lg + (size_t)(t - tb0) * E;
     float v[NV];
     uint32_t taken = 0;
@@ -400,10 +413,10 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   }
     __syncthreads();  // the staging buffer is reused by the next group of tokens
   }
-  for (int e = tid; e < E; e += kRouterThreads) s_cnt[e] = 0;
+  for (int e = tid; e < E; e += NT) s_cnt[e] = 0;
   __syncthreads();
   const int nas = B * k;
-  for (int i = tid; i < nas; i += kRouterThreads) atomicAdd(&s_cnt[s_ids[i]], 1);
+  for (int i = tid; i < nas; i += NT) atomicAdd(&s_cnt[s_ids[i]], 1);
   __syncthreads();
 
   // Exclusive scans of counts and of units per expert over E (<= 1024 =
@@ -418,8 +431,8 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
     fsum += f4[i];
   }
   int ctot, ftot;
-  int cbase = block_exclusive_scan(csum, s_warp, ctot);
-  int fbase = block_exclusive_scan(fsum, s_warp, ftot);
+  int cbase = block_exclusive_scan<NT>(csum, s_warp, ctot);
+  int fbase = block_exclusive_scan<NT>(fsum, s_warp, ftot);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int e = tid * 4 + i;
@@ -445,7 +458,7 @@ __global__ void __launch_bounds__(kRouterThreads, 1) router_topk_kernel(const __
   // walks the tokens in order, lane j placing slot j, with a per-expert fill
   // counter (the ids of one token are distinct, so no two lanes of a step
   // share a counter); each expert's assignments end up ordered by token.
-  for (int e = tid; e < E; e += kRouterThreads) s_cnt[e] = 0;
+  for (int e = tid; e < E; e += NT) s_cnt[e] = 0;
   __syncthreads();
   if (warp == 0) {
     for (int t = 0; t < B; ++t) {

@@ -134,14 +134,26 @@ def test_repeated_calls_are_consistent(tiny):
     oracle_check(tiny.wts, 2, x, o2, i2, w2)
 
 
-def test_host_buffer_entry_point(tiny):
+@pytest.mark.parametrize("kind,B", [("pinned", 4), ("pageable", 4), ("mixed", 4), ("pinned", 13)])
+def test_host_buffer_entry_point(tiny, kind, B):
+    # pinned (mapped) outputs are stored by the kernels directly; pageable or
+    # mixed ones go through device staging and copies
     wts = tiny.wts
-    x = margin_x(4, synth.TINY.hidden, wts, 2, seed=8).cpu().pin_memory()
-    out = torch.empty_like(x).pin_memory()
-    ids = torch.empty(4, 2, dtype=torch.int32).pin_memory()
-    w = torch.empty(4, 2, dtype=torch.float32).pin_memory()
-    tiny.blk.forward_host(x, wts.router_w, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, out, ids, w)
-    oracle_check(wts, 2, x, out, ids, w)
+    x = margin_x(B, synth.TINY.hidden, wts, 2, seed=8 + B).cpu()
+    out = torch.empty_like(x)
+    ids = torch.empty(B, 2, dtype=torch.int32)
+    w = torch.empty(B, 2, dtype=torch.float32)
+    if kind == "pinned":
+        x, out, ids, w = x.pin_memory(), out.pin_memory(), ids.pin_memory(), w.pin_memory()
+    elif kind == "mixed":
+        out = out.pin_memory()
+    for _ in range(2):
+        out.fill_(float("nan"))
+        ids.fill_(-1)
+        w.fill_(float("nan"))
+        tiny.blk.forward_host(x, wts.router_w, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, out, ids, w)
+        oracle_check(wts, 2, x, out, ids, w)
+    assert tiny.blk.status() == MOE_OK
 
 
 def _graph_alternating(run, xa, xb, replays=20):
