@@ -47,18 +47,18 @@
 // change chunks at about the same time, those stalls line up into dips of
 // the whole GPU's bandwidth.
 //
-// Panels.  Each matrix is cut into column panels and K-row stages.  A
-// consumer thread keeps at most 128 fp32 accumulators, so panel columns x
-// token tiles is bounded; a unit with n tokens uses the widest panel its
-// token count allows --
+// Panels.  Each matrix is cut into column panels and K-row stages of 64 KB
+// of weights.  A unit with n tokens takes the panel of its token class, the
+// narrower the more token tiles it has, so that a consumer warp's columns x
+// token tiles -- its accumulators -- stay the same in every class:
 //   class 0: n <=  8 : 2048 local columns, 16-row stages (1 token tile)
-//   class 1: n <= 16 : 2048 local columns, 16-row stages (2 token tiles)
-//   class 2: n <= 32 : 1024 local columns, 32-row stages (4 token tiles)
-// -- every stage is 64 KB of weights.  A launch is compiled for the largest
-// class its batch can produce (KC), so batches of <= 8 tokens run code that
-// holds only 32 accumulators per thread (with 16 consumer warps).  UP panels
-// pair gate columns [c0, c0 + LW/2) with up columns [I + c0, ...), so a panel
-// holds both halves of its SwiGLU.
+//   class 1: n <= 16 : 1024 local columns, 32-row stages (2 token tiles)
+//   class 2: n <= 32 :  512 local columns, 64-row stages (4 token tiles)
+// -- 16 consumer warps, each with 32 fp32 accumulators, in every instance.
+// A launch is compiled for the largest class its batch can produce (KC), so
+// small batches carry no code for the wider classes.  UP panels pair gate
+// columns [c0, c0 + LW/2) with up columns [I + c0, ...), so a panel holds
+// both halves of its SwiGLU.
 //
 // Data movement.  One producer warp fills a shared-memory ring of 64 KB
 // stages, guarded by mbarriers, with TMA (no multicast, L2 evict-first):
