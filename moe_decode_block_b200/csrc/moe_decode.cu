@@ -274,10 +274,10 @@ int router_threads_for(int n_experts) {
 
 // CTAs for the shared expert when it runs beside the routed experts: its
 // share of the forward's weight bytes (routed share estimated for uniform
-// routing, E * (1 - (1 - k/E)^B) distinct experts), scaled up when the batch
-// puts the shared expert in a narrow-panel class whose smaller row copies
-// stream more slowly per SM.  The routed kernel gets the remaining SMs, so the
-// two grids never wait for each other's SMs.
+// routing, E * (1 - (1 - k/E)^B) distinct experts), weighted up for the wider
+// token classes, whose stages take the consumers longer per byte (empirical
+// factors; only this two-stream plan uses them).  The routed kernel gets the
+// remaining SMs, so the two grids never wait for each other's SMs.
 int shared_grid(const moe_decode_ctx* h, int batch) {
   if (h->grid_shared > 0) return h->grid_shared;
   const moe_decode_shapes& s = h->s;
