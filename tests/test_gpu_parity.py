@@ -86,6 +86,25 @@ def test_tiny_odd_shapes_several_panels_and_ragged_steps(plan):
         oracle_check(wts, s.top_k, x, out, ids, w)
 
 
+@pytest.mark.parametrize("H,E,k,B", [
+    (256, 8, 8, 64),     # k == E: every token selects every expert (64 tokens -> two units each)
+    (256, 64, 12, 8),    # k > 8: the router's k-round argmax path (64-expert instance)
+    (512, 64, 32, 64),   # the largest top-k: 2048 assignments, experts above 32 tokens split
+    (256, 384, 16, 8),   # k > 8 on the 384-expert router instance
+])
+def test_wide_top_k_and_every_expert_selected(H, E, k, B):
+    s = synth.BlockShape(hidden=H, n_experts=E, top_k=k, inter=128, shared_inter=128, n_shared=1)
+    wts = synth.make_weights(s, seed=5, device="cuda")
+    run = Run(s, wts, max_batch=B)
+    try:
+        x = margin_x(B, s.hidden, wts, k, seed=50 + k)
+        out, ids, w = run.forward(x)
+        oracle_check(wts, k, x, out, ids, w)
+        assert run.blk.status() == MOE_OK
+    finally:
+        run.blk.close()
+
+
 def test_zero_down_weights_give_the_input_bitwise(tiny):
     wts = tiny.wts
     z2 = torch.zeros_like(wts.w2)
