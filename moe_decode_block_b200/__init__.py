@@ -211,7 +211,9 @@ class MoEDecode:
 
     def forward_host(self, x_host, router_w, w13, w2, shared_w13, shared_w2, out_host, ids_host, w_host,
                      batch: Optional[int] = None, stream_main=None, stream_aux=None):
-        """Host-buffer variant: copies x in and out/ids/w back, synchronising stream_main."""
+        """Host-buffer variant, synchronising stream_main: x is copied in; out/ids/w
+        are stored by the kernels directly when all three are pinned (mapped)
+        host tensors, else staged on the device and copied back."""
         import torch
         if batch is None:
             batch = x_host.shape[0]
