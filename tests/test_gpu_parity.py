@@ -91,6 +91,8 @@ def test_tiny_odd_shapes_several_panels_and_ragged_steps(plan):
     (256, 64, 12, 8),    # k > 8: the router's k-round argmax path (64-expert instance)
     (512, 64, 32, 64),   # the largest top-k: 2048 assignments, experts above 32 tokens split
     (256, 384, 16, 8),   # k > 8 on the 384-expert router instance
+    (256, 1024, 8, 64),  # the largest expert count (the 256-thread router instance), top-8 path
+    (256, 1024, 12, 8),  # ... and its k-round path
 ])
 def test_wide_top_k_and_every_expert_selected(H, E, k, B):
     s = synth.BlockShape(hidden=H, n_experts=E, top_k=k, inter=128, shared_inter=128, n_shared=1)
