@@ -54,6 +54,10 @@ def _load():
         lib.oracle_router.restype = I
         lib.oracle_block.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P]
         lib.oracle_block.restype = I
+        lib.oracle_expert_outputs.argtypes = [P, I, I, P, P, I, I, P, P]
+        lib.oracle_expert_outputs.restype = I
+        lib.oracle_combine.argtypes = [P, P, P, P, I, I, I, P]
+        lib.oracle_combine.restype = I
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = I
         _lib = lib
@@ -129,6 +133,51 @@ def block(x, ids, w, w13: Sequence, w2: Sequence, sw13=None, sw2=None, n_experts
     _check(lib.oracle_block(_ptr(x), _ptr(ids), _ptr(w), arr13, arr2, _ptr(sw13), _ptr(sw2),
                             B, H, E, k, inter, Is, n_shared, _ptr(out)), "oracle_block")
     del keep
+    return out
+
+
+def expert_outputs(x, w13e, w2e, rows):
+    """Step 5 for one expert (C oracle): y [len(rows), H] f64, row i the
+    SwiGLU MLP of token rows[i] through that expert's w13e [H,2I], w2e [I,H]."""
+    lib = _load()
+    x = _u16(x)
+    B, H = x.shape
+    w13e = _u16(w13e)
+    w2e = _u16(w2e)
+    I = w13e.shape[1] // 2
+    assert w13e.shape == (H, 2 * I) and w2e.shape == (I, H)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    y = np.zeros((len(rows), H), np.float64)
+    _check(lib.oracle_expert_outputs(_ptr(x), B, H, _ptr(w13e), _ptr(w2e), I, len(rows), _ptr(rows), _ptr(y)),
+           "oracle_expert_outputs")
+    return y
+
+
+def block_streamed(x, ids, w, fetch_expert, sw13=None, sw2=None):
+    """Steps 5-7 like ``block``, holding one expert's weights at a time:
+    ``fetch_expert(e)`` returns (w13[e], w2[e]) as bf16 bit arrays and is
+    called once per distinct selected expert, in ascending id order.  Each
+    expert's MLP is evaluated for the tokens that chose it, the per-assignment
+    outputs are kept, and the sum of step 7 is taken in the same order as
+    ``block`` (residual, then j = 0..k-1, then the shared expert), so the
+    result is bitwise equal to ``block``'s."""
+    lib = _load()
+    x = _u16(x)
+    B, H = x.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    k = ids.shape[1] if ids.ndim == 2 else 0
+    y = np.zeros((B, k, H), np.float64)
+    for e in sorted(set(ids.ravel().tolist())):
+        bj = np.argwhere(ids == e)  # (token, slot) pairs that chose e
+        a13, a2 = fetch_expert(e)
+        y[bj[:, 0], bj[:, 1]] = expert_outputs(x, a13, a2, bj[:, 0])
+        del a13, a2
+    s = None
+    if sw13 is not None:
+        s = expert_outputs(x, sw13, sw2, np.arange(B))
+    out = np.zeros((B, H), np.float64)
+    _check(lib.oracle_combine(_ptr(x), _ptr(w), _ptr(y), _ptr(s), B, H, k, _ptr(out)), "oracle_combine")
     return out
 
 

@@ -188,6 +188,56 @@ done:
   return rc;
 }
 
+/* Step 5 (or 6) for one expert and a list of tokens, the building block of
+ * the expert-at-a-time driver: y[i, :] = (silu(g) * u) . W2 for token
+ * rows[i] of x, with W13 [H,2I], W2 [I,H] that expert's weights. */
+int oracle_expert_outputs(const uint16_t* x, int B, int H, const uint16_t* W13,
+                          const uint16_t* W2, int I, int n, const int32_t* rows,
+                          double* y) {
+  if (B < 0 || H <= 0 || I <= 0 || n < 0) return ORACLE_BAD_ARG;
+  if (n == 0) return ORACLE_OK;
+  if (!x || !W13 || !W2 || !rows || !y) return ORACLE_BAD_ARG;
+  double* xb = (double*)malloc(sizeof(double) * (size_t)H);
+  double* gu = (double*)malloc(sizeof(double) * 2 * (size_t)I);
+  double* a = (double*)malloc(sizeof(double) * (size_t)I);
+  int rc = ORACLE_OK;
+  if (!xb || !gu || !a) {
+    rc = ORACLE_NO_MEMORY;
+    goto done;
+  }
+  for (int i = 0; i < n; ++i) {
+    const int b = rows[i];
+    if (b < 0 || b >= B) { rc = ORACLE_BAD_ARG; goto done; }
+    for (int h = 0; h < H; ++h) xb[h] = bf16_bits_to_double(x[(size_t)b * H + h]);
+    swiglu_mlp(xb, W13, W2, H, I, gu, a, y + (size_t)i * H);
+  }
+done:
+  free(xb); free(gu); free(a);
+  return rc;
+}
+
+/* Step 7 from per-assignment expert outputs: out_b = x_b + sum_j w_j y[b,j]
+ * (+ s_b), with y [B,k,H] and s [B,H] (NULL: no shared expert) -- the same
+ * additions, in the same order, as oracle_block. */
+int oracle_combine(const uint16_t* x, const double* w, const double* y,
+                   const double* s, int B, int H, int k, double* out) {
+  if (B < 0 || H <= 0 || k < 0) return ORACLE_BAD_ARG;
+  if (B == 0) return ORACLE_OK;
+  if (!x || !out || (k > 0 && (!w || !y))) return ORACLE_BAD_ARG;
+  for (int b = 0; b < B; ++b) {
+    double* ob = out + (size_t)b * H;
+    for (int h = 0; h < H; ++h) ob[h] = bf16_bits_to_double(x[(size_t)b * H + h]);
+    for (int j = 0; j < k; ++j) {
+      const double wj = w[(size_t)b * k + j];
+      const double* yj = y + ((size_t)b * k + j) * H;
+      for (int h = 0; h < H; ++h) ob[h] += wj * yj[h];
+    }
+    if (s)
+      for (int h = 0; h < H; ++h) ob[h] += s[(size_t)b * H + h];
+  }
+  return ORACLE_OK;
+}
+
 /* Steps 1-7. */
 int oracle_moe_forward(const uint16_t* x, const uint16_t* router_w, const float* bias,
                        const uint16_t* const* w13, const uint16_t* const* w2,

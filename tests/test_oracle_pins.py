@@ -335,3 +335,39 @@ def test_tiny_config_inputs_through_both_oracles():
     np.testing.assert_allclose(oc, on, rtol=1e-12, atol=1e-12)
     assert abs(wc.sum() - 1) < 1e-12
     assert oracle.topk_margin(lc, 2)[0] > 0
+
+
+# ------------------------------------------- expert-at-a-time driver ---
+
+@pytest.mark.parametrize("B,k,shared", [(1, 2, True), (7, 3, True), (16, 8, False), (33, 16, True)])
+def test_streamed_block_is_bitwise_the_block(B, k, shared):
+    # block_streamed evaluates each selected expert for the tokens that chose
+    # it and sums in block's order, so it must equal block() bit for bit; it
+    # fetches every selected expert exactly once, in ascending id order, and
+    # nothing else
+    d = rand_block(B=B, H=48, E=24, k=k, I=16, Is=24, seed=40 + B)
+    _, ids, w = oracle.router(d["x"], d["router_w"], k, None)
+    sw13, sw2 = (d["sw13"], d["sw2"]) if shared else (None, None)
+    ref = oracle.block(d["x"], ids, w, d["w13"], d["w2"], sw13, sw2)
+    fetched = []
+
+    def fetch(e):
+        fetched.append(e)
+        return d["w13"][e], d["w2"][e]
+
+    got = oracle.block_streamed(d["x"], ids, w, fetch, sw13, sw2)
+    assert np.array_equal(got, ref)
+    assert fetched == sorted(set(ids.ravel().tolist()))
+
+
+def test_expert_outputs_is_one_swiglu_mlp_per_row():
+    # one expert's outputs for a row list equal the block of a top-1 routing
+    # to that expert with the residual taken away (weight 1, no shared)
+    d = rand_block(B=5, H=32, E=8, k=1, I=8, Is=8, seed=9)
+    rows = np.array([4, 0, 2, 2], dtype=np.int32)
+    y = oracle.expert_outputs(d["x"], d["w13"][3], d["w2"][3], rows)
+    ids = np.full((5, 1), 3, np.int32)
+    full = oracle.block(d["x"], ids, np.ones((5, 1)), d["w13"], d["w2"])
+    resid = d["x"].astype(np.uint32) << 16
+    xr = resid.view(np.float32).astype(np.float64)
+    np.testing.assert_allclose(y, (full - xr)[rows], rtol=0, atol=1e-12)
