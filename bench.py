@@ -20,6 +20,14 @@ per step x steps x ranks / max-over-ranks device time.  Under torchrun every
 rank runs an independent replica of the block on its own batch (weak scaling,
 no collective on the data path).
 
+At N=1 the same run also times the other graded configurations on the same
+weight set (full-size batch 8 and 64, Zipf-routed batch 32: the `configs`
+object), and rank 0 checks every timed forward against the fp64 oracle (ids
+exact, weights within 1e-5, outputs within 2e-2 * rms): the `parity` key; a
+failed check makes the run exit non-zero.  Token inputs carry a top-k logit
+margin >= 1e-3: each row's redraw counter comes from
+tests/golden/bench_inputs.json (written by tests/golden/make_bench_inputs.py).
+
 --impl reference times the fp64 CPU oracle on the host cores instead.
 """
 from __future__ import annotations
@@ -39,6 +47,11 @@ if ROOT not in sys.path:
 
 METRIC = "MoE decode block µs and achieved HBM GB/s vs B200 peak, batch 1–64, 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # the nominal B200 HBM3e figure, for context
+CONFIG_WORKLOADS = ("full_b8", "full_b64", "zipf_b32")
+OUT_RTOL = 2e-2
+W_ATOL = 1e-5
+INPUTS_JSON = os.path.join(ROOT, "tests", "golden", "bench_inputs.json")
 
 
 def parse_args():
@@ -53,7 +66,31 @@ def parse_args():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--two-stream", action="store_true",
                    help="time the plan with the shared expert on the aux stream (MOE_FLAG_TWO_STREAM)")
+    p.add_argument("--no-configs", action="store_true", help="skip the other graded configurations")
+    p.add_argument("--config-steps", type=int, default=200, help="timed graph replays per extra configuration")
+    p.add_argument("--no-parity", action="store_true", help="skip the oracle check of the timed forwards")
     return p.parse_args()
+
+
+def x_attempts(workload: str, x_seed: int):
+    """Per-row redraw counters giving this workload's x (drawn from x_seed) a
+    top-k logit margin, or None when none are stored for it."""
+    try:
+        with open(INPUTS_JSON) as f:
+            d = json.load(f)
+        return d["workloads"][workload][str(x_seed)]
+    except Exception:
+        return None
+
+
+def make_inputs(wl, seed: int, x_seed: int, dev):
+    """Weights (router drawn on the host generator, the rest on the device)
+    and the margin-checked x of a workload.  Returns (weights, x, margin)."""
+    from moe_decode_block_b200 import synth
+    wts = synth.make_weights(wl.shape, seed=seed, device=dev, routing=wl.routing, router_device="cpu")
+    att = x_attempts(wl.name, x_seed) if seed == 0 else None
+    x = synth.make_x(wl.batch, wl.shape.hidden, seed=x_seed, attempts=att).to(dev)
+    return wts, x, ("top-k margin >= 1e-3 (stored redraw counters)" if att is not None else "unchecked")
 
 
 def peaks():
@@ -226,9 +263,13 @@ def time_oracle(wl, inp, bytes_step, min_seconds=10.0, max_runs=30, warmup=1, ma
     import oracle
     k = wl.shape.top_k
 
+    last = {}
+
     def one():
         _, ids, w = oracle.router(inp["x"], inp["R"], k, inp["bias"])
-        oracle.block(inp["x"], ids, w, inp["h13"], inp["h2"], inp["sw13"], inp["sw2"], n_experts=wl.shape.n_experts)
+        out = oracle.block(inp["x"], ids, w, inp["h13"], inp["h2"], inp["sw13"], inp["sw2"],
+                           n_experts=wl.shape.n_experts)
+        last.update(out=out, ids=ids, w=w)
 
     done_warmup = 0
     t_w = time.perf_counter()
@@ -249,6 +290,7 @@ def time_oracle(wl, inp, bytes_step, min_seconds=10.0, max_runs=30, warmup=1, ma
         if max_seconds is not None and el >= max_seconds:
             break
     per = statistics.median(times)
+    time_oracle.last = last
     return bytes_step / per / 1e9, per, len(times), oracle.num_threads(), done_warmup
 
 
@@ -267,8 +309,8 @@ def run_reference(args):
     # drawing 34 GB of full-size weights on the host is slow); only the
     # touched experts are copied to the host for the oracle
     gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
-    wts = synth.make_weights(wl.shape, seed=args.seed, device=gen_dev, routing=wl.routing)
-    x = synth.make_x(wl.batch, wl.shape.hidden, seed=args.seed)
+    wts, x, _ = make_inputs(wl, args.seed, args.seed, gen_dev)
+    x = x.cpu()
     import oracle
     bias = None if wts.router_bias is None else wts.router_bias.float().cpu().numpy()
     _, ids, _ = oracle.router(synth.bf16_bits(x), synth.bf16_bits(wts.router_w), wl.shape.top_k, bias)
@@ -304,6 +346,40 @@ def _config_dict(wl, graph=True):
             "parallelism": "replicas (one independent block per GPU)"}
 
 
+def check_against_oracle(wts, x, out, ids, w, k, ref=None):
+    """The timed forward's results against the fp64 oracle (ids exact,
+    weights within W_ATOL, outputs within OUT_RTOL * rms over every element).
+    ref: the oracle's (out, ids, w) for these inputs if already computed;
+    otherwise the oracle is run here, one selected expert at a time.
+    Returns a small dict with "ok"."""
+    import numpy as np
+
+    import oracle
+    from moe_decode_block_b200 import synth
+    xb = synth.bf16_bits(x)
+    if ref is None:
+        bias = None if wts.router_bias is None else wts.router_bias.float().cpu().numpy()
+        _, o_ids, o_w = oracle.router(xb, synth.bf16_bits(wts.router_w), k, bias)
+
+        def fetch(e):
+            return synth.bf16_bits(wts.w13[e]), synth.bf16_bits(wts.w2[e])
+
+        o_out = oracle.block_streamed(xb, o_ids, o_w, fetch, synth.bf16_bits(wts.shared_w13),
+                                      synth.bf16_bits(wts.shared_w2))
+    else:
+        o_out, o_ids, o_w = ref
+    g_ids = ids.cpu().numpy()
+    g_w = w.cpu().numpy().astype(np.float64)
+    g_out = out.float().cpu().numpy()
+    ids_ok = bool(np.array_equal(g_ids, o_ids))
+    w_err = float(np.max(np.abs(g_w - o_w), initial=0.0))
+    err = float(np.max(np.abs(g_out - o_out), initial=0.0)) if np.all(np.isfinite(g_out)) else float("inf")
+    rms = float(np.sqrt(np.mean(o_out ** 2)))
+    ok = ids_ok and w_err <= W_ATOL and err <= OUT_RTOL * rms
+    return {"ok": ok, "ids_exact": ids_ok, "max_w_err": w_err, "max_out_err": err,
+            "tol": OUT_RTOL * rms, "rows": int(x.shape[0])}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -329,77 +405,83 @@ def run_ours(args):
     wl = synth.WORKLOADS[args.config]
     s = wl.shape
     B = wl.batch
-    wts = synth.make_weights(s, seed=args.seed, device=dev, routing=wl.routing)
-    x = synth.make_x(B, s.hidden, seed=args.seed + 1000 * rank).to(dev)
-    blk = MoEDecode(s.hidden, s.n_experts, s.top_k, s.inter, s.shared_inter, n_shared=s.n_shared,
-                    max_batch=max(B, 1), router_bias=wts.router_bias, two_stream=args.two_stream)
-    out = torch.empty_like(x)
-    ids = torch.empty(B, s.top_k, dtype=torch.int32, device=dev)
-    w = torch.empty(B, s.top_k, dtype=torch.float32, device=dev)
+    wts, x, margin = make_inputs(wl, args.seed, args.seed + 1000 * rank, dev)
     main = torch.cuda.Stream()
     aux = torch.cuda.Stream()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush_buf = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
     flush_sum = torch.empty((), dtype=torch.float32, device=dev)
 
-    class _Flush:
+    def flush():
         """Write a 2x-L2 buffer, then read it back: the write evicts every
         weight line; the read leaves L2 holding clean lines, so the timed step
         pays no write-back of the flush's dirty lines."""
+        flush_buf.zero_()
+        torch.sum(flush_buf, dim=0, out=flush_sum)
 
-        @staticmethod
-        def zero_():
-            flush_buf.zero_()
-            torch.sum(flush_buf, dim=0, out=flush_sum)
+    class Case:
+        """One handle + buffers + a CUDA graph of one forward of a workload."""
 
-    flush = _Flush()
-    fargs = (x, wts.router_w, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, out, ids, w)
+        def __init__(self, wl_, wts_, x_, two_stream):
+            sh = wl_.shape
+            self.wl, self.wts, self.x = wl_, wts_, x_
+            self.blk = MoEDecode(sh.hidden, sh.n_experts, sh.top_k, sh.inter, sh.shared_inter, n_shared=sh.n_shared,
+                                 max_batch=max(wl_.batch, 1), router_bias=wts_.router_bias, two_stream=two_stream)
+            self.out = torch.empty_like(x_)
+            self.ids = torch.empty(wl_.batch, sh.top_k, dtype=torch.int32, device=dev)
+            self.w = torch.empty(wl_.batch, sh.top_k, dtype=torch.float32, device=dev)
+            self.fargs = (x_, wts_.router_w, wts_.w13, wts_.w2, wts_.shared_w13, wts_.shared_w2, self.out, self.ids,
+                          self.w)
+            with torch.cuda.stream(main):
+                self.blk.forward(*self.fargs, stream_main=main, stream_aux=aux)
+            main.synchronize()
+            if self.blk.status() != 0:
+                raise RuntimeError(f"device status not OK after the first forward of {wl_.name}")
+            self.bstep, self.distinct = bytes_per_step(sh, self.ids.cpu().numpy(), wl_.batch)
+            self.kernels_per_step = self.blk.stats()["last_kernels"]
+            self.g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g, stream=main):
+                self.blk.forward(*self.fargs, stream_main=torch.cuda.current_stream(), stream_aux=aux)
 
-    with torch.cuda.stream(main):
-        blk.forward(*fargs, stream_main=main, stream_aux=aux)
-    main.synchronize()
-    if blk.status() != 0:
-        raise RuntimeError("device status not OK after the first forward")
-    bstep, distinct = bytes_per_step(s, ids.cpu().numpy(), B)
-    kernels_per_step = blk.stats()["last_kernels"]
+        def timed(self, steps, warmup):
+            """Graph replays with L2 flushed before each; per-step ms (events on
+            the launching stream around the replay only) and the clocks seen."""
+            with torch.cuda.stream(main):
+                for _ in range(warmup):
+                    flush()
+                    self.g.replay()
+            torch.cuda.synchronize()
+            sampler = ClockSampler(dev.index)
+            sampler.start()
+            time.sleep(0.2)
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            w0 = time.perf_counter()
+            starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+            ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+            with torch.cuda.stream(main):
+                for i in range(steps):
+                    flush()
+                    starts[i].record(main)
+                    self.g.replay()
+                    ends[i].record(main)
+            torch.cuda.synchronize()
+            w1 = time.perf_counter()
+            if world > 1:
+                torch.distributed.barrier()
+            clocks = sampler.stop()
+            return [a.elapsed_time(b) for a, b in zip(starts, ends)], clocks, (w1 - w0) * 1e3
 
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=main):
-        blk.forward(*fargs, stream_main=torch.cuda.current_stream(), stream_aux=aux)
+        def close(self):
+            del self.g
+            self.blk.close()
 
-    def timed_loop(n, step_fn):
-        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        with torch.cuda.stream(main):
-            for i in range(n):
-                flush.zero_()
-                starts[i].record(main)
-                step_fn()
-                ends[i].record(main)
-        return starts, ends
-
-    # ---- warm-up
-    with torch.cuda.stream(main):
-        for _ in range(args.warmup):
-            flush.zero_()
-            g.replay()
-    torch.cuda.synchronize()
+    head = Case(wl, wts, x, args.two_stream)
+    blk, fargs, bstep, distinct = head.blk, head.fargs, head.bstep, head.distinct
 
     # ---- headline: graph replays, L2 flushed before each step
-    sampler = ClockSampler(dev.index)
-    sampler.start()
-    time.sleep(0.2)
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    starts, ends = timed_loop(args.steps, g.replay)
-    torch.cuda.synchronize()
-    wall1 = time.perf_counter()
-    if world > 1:
-        torch.distributed.barrier()
-    clocks = sampler.stop()
-    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    step_ms, clocks, bracket_ms = head.timed(args.steps, args.warmup)
     value, total_ms, all_bytes = aggregate_over_ranks(float(sum(step_ms)), bstep, args.steps, dev, world)
     ms_per_step = total_ms / args.steps
 
@@ -410,7 +492,7 @@ def run_ours(args):
     nb = min(args.steps, 200)
     with torch.cuda.stream(main):
         for i in range(nb + 5):
-            flush.zero_()
+            flush()
             blk.forward(*fargs, stream_main=main, stream_aux=aux)
             main.synchronize()
             aux.synchronize()
@@ -435,6 +517,7 @@ def run_ours(args):
     exp_gbs = exp_bytes / (kern_us["experts"] * 1e-6) / 1e9
     kname = "expert_mlp_routed" if args.two_stream else "expert_mlp"
     traffic = ncu_traffic(kname, wl.name)
+    block_gbs = bstep / (ms_per_step * 1e-3) / 1e9
     roofline = {"bound": "hbm",
                 "kernel": "expert_mlp_kernel<routed only>" if args.two_stream
                 else "expert_mlp_kernel<shared + routed>",
@@ -442,7 +525,9 @@ def run_ours(args):
                 "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(exp_gbs / peak, 4),
                 "traffic": traffic, "algorithmic_bytes_per_launch": exp_bytes,
                 "launch_us": kern_us["experts"],
-                "block_frac": round((bstep / (ms_per_step * 1e-3) / 1e9) / peak, 4)}
+                "block_frac": round(block_gbs / peak, 4),
+                "frac_of_nominal_8tbs": round(exp_gbs / NOMINAL_HBM_GBS, 4),
+                "block_frac_of_nominal_8tbs": round(block_gbs / NOMINAL_HBM_GBS, 4)}
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -455,7 +540,7 @@ def run_ours(args):
         times = []
         with torch.cuda.stream(main):
             for i in range(ne + 5):
-                flush.zero_()
+                flush()
                 main.synchronize()
                 t0 = time.perf_counter()
                 blk.forward_host(xh, wts.router_w, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, oh, ih, wh,
@@ -474,37 +559,87 @@ def run_ours(args):
                "api": "moe_decode_forward_host (pinned host buffers: x copied in; out, topk_ids, topk_w "
                       "stored into them by the kernels; synchronous)"}
 
-    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N == 1)
+    # ---- the other graded configurations, same weights (N == 1)
+    configs = None
+    cases = []
+    if world == 1 and not args.no_configs and s == synth.FULL:
+        configs = {}
+        for name in CONFIG_WORKLOADS:
+            if name == wl.name:
+                continue
+            cwl = synth.WORKLOADS[name]
+            cw = wts
+            if cwl.routing != wl.routing:
+                bias = synth.zipf_log_prior(s.n_experts, args.seed, dev) if cwl.routing == "zipf" else None
+                cw = synth.BlockWeights(wts.router_w, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, bias)
+            att = x_attempts(name, args.seed) if args.seed == 0 else None
+            cx = synth.make_x(cwl.batch, s.hidden, seed=args.seed, attempts=att).to(dev)
+            case = Case(cwl, cw, cx, args.two_stream)
+            ms, cclk, _ = case.timed(args.config_steps, 20)
+            us = 1e3 * statistics.mean(ms)
+            gbs = case.bstep / (us * 1e-6) / 1e9
+            configs[name] = {"batch": cwl.batch, "routing": cwl.routing, "distinct_experts": case.distinct,
+                             "bytes_per_step": case.bstep, "us_per_block": round(us, 2),
+                             "us_p10": round(1e3 * float(np.percentile(ms, 10)), 2),
+                             "us_p90": round(1e3 * float(np.percentile(ms, 90)), 2),
+                             "GB/s": round(gbs, 1), "frac_of_measured_peak": round(gbs / peak, 4),
+                             "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+                             "tokens_per_s": round(cwl.batch / (us * 1e-6), 1), "steps": args.config_steps,
+                             "margin": "top-k margin >= 1e-3 (stored redraw counters)" if att is not None
+                             else "unchecked", "clocks": cclk}
+            cases.append(case)
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N == 1); its
+    # last run is the oracle output the headline forward is checked against
     cpu = None
+    oracle_ref = None
     if world == 1 and not args.no_cpu_baseline:
-        inp = host_oracle_inputs(wl, wts, x, ids.cpu().numpy())
+        inp = host_oracle_inputs(wl, wts, x, head.ids.cpu().numpy())
         gbs, per, runs, threads, _ = time_oracle(wl, inp, bstep, min_seconds=10.0, max_runs=30)
+        last = time_oracle.last
+        oracle_ref = (last["out"], last["ids"], last["w"])
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                "sample": f"{runs} full forwards of the {wl.name} block (router + {distinct} routed + shared "
                          f"expert MLPs) by the fp64 C oracle, >= 10 s of CPU work, median "
                          f"{per * 1e3:.1f} ms per block"}
 
+    # ---- parity of every timed forward against the oracle (rank 0)
+    parity = None
+    if rank == 0 and not args.no_parity:
+        parity = {"bar": f"ids exact, |w - oracle| <= {W_ATOL}, max|out - oracle| <= {OUT_RTOL} * rms(oracle out)",
+                  wl.name: check_against_oracle(wts, x, head.out, head.ids, head.w, s.top_k, oracle_ref)}
+        for case in cases:
+            parity[case.wl.name] = check_against_oracle(case.wts, case.x, case.out, case.ids, case.w, s.top_k)
+        parity["ok"] = all(v["ok"] for k, v in parity.items() if isinstance(v, dict))
+        if configs:
+            for name in configs:
+                configs[name]["parity"] = "ok" if parity[name]["ok"] else "FAIL"
+
     status = blk.status()
+    parity_ok = parity is None or parity["ok"]
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(_config_dict(wl), plan="two_stream" if args.two_stream else "default"),
+            "config": dict(_config_dict(wl), plan="two_stream" if args.two_stream else "default", inputs=margin),
             "us_per_block": round(ms_per_step * 1e3, 2), "tokens_per_s": round(B * 1e3 / ms_per_step, 1),
             "bytes_per_step": bstep, "distinct_experts": distinct,
             "roofline": roofline, "kernels_us": kern_us, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": kernels_per_step * args.steps, "kernels_per_step": kernels_per_step,
-            "clocks": clocks, "bracket_ms_incl_flush": round((wall1 - wall0) * 1e3, 2),
+            "parity": "ok" if parity_ok and parity is not None else ("FAIL" if not parity_ok else None),
+            "parity_detail": parity, "configs": configs,
+            "gpu_launches": head.kernels_per_step * args.steps, "kernels_per_step": head.kernels_per_step,
+            "clocks": clocks, "bracket_ms_incl_flush": round(bracket_ms, 2),
             "device_status": status,
         }
         print(json.dumps(line), flush=True)
-    del g
-    blk.close()
+    for case in cases:
+        case.close()
+    head.close()
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
-    return 0
+    return 0 if parity_ok and status == 0 else 1
 
 
 def main():

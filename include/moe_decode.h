@@ -81,9 +81,9 @@ extern "C" {
  * router_bias (optional) is a device float32 [n_experts] added to the router
  * logits before softmax and selection; NULL means no bias.  It is read by
  * every forward (the pointer is kept, the data is not copied).
- * flags: any combination of MOE_FLAG_TWO_STREAM (see the top of this file)
- * and MOE_FLAG_TCGEN05 (below); other bits are rejected with
- * MOE_ERR_UNSUPPORTED_SHAPE.
+ * flags: any combination of MOE_FLAG_TWO_STREAM (see the top of this file),
+ * MOE_FLAG_TCGEN05 and MOE_FLAG_TEST_HOLD_PANEL (below); other bits are
+ * rejected with MOE_ERR_UNSUPPORTED_SHAPE.
  */
 #define MOE_FLAG_TWO_STREAM 1u
 /*
@@ -97,6 +97,16 @@ extern "C" {
  * those from one thread takes about as long as HBM takes to deliver the stage.
  */
 #define MOE_FLAG_TCGEN05 2u
+/*
+ * MOE_FLAG_TEST_HOLD_PANEL (testing only): the handle's first forward
+ * withholds the publication of one routed up-projection panel, so the
+ * down-projection stages that need it wait until their bounded wait gives
+ * up.  That forward's outputs are wrong and moe_decode_get_status reports
+ * MOE_ERR_DEVICE_TIMEOUT; later forwards of the handle are normal.  Used,
+ * with a short moe_decode_set_wait_limit, to test the device-side timeout
+ * path without faulting or hanging the GPU.
+ */
+#define MOE_FLAG_TEST_HOLD_PANEL 4u
 typedef struct moe_decode_shapes {
   int32_t hidden;
   int32_t n_experts;
@@ -112,20 +122,28 @@ typedef struct moe_decode_shapes {
 typedef struct moe_decode_ctx* moe_decode_t;
 
 /*
- * Per-handle counters (host side), filled by moe_decode_get_stats.
+ * Per-handle counters, filled by moe_decode_get_stats.  Host side:
  *   forwards          : successful forwards enqueued by this handle
  *   kernels_launched  : kernels enqueued by this handle since creation
  *   last_kernels      : kernels enqueued by the last forward (default plan:
  *                       3; MOE_FLAG_TWO_STREAM: 4, or 3 without a shared
  *                       expert)
  *   last_token_tiles  : token tiles of 8 the expert kernels were prepared for
- *                       in the last forward (ceil(batch / 8))
+ *                       in the last forward (ceil(min(batch, 32) / 8))
+ * Device side (counted by the expert kernels as they run, cumulative since
+ * moe_decode_init, graph replays included):
+ *   stages_up[c], stages_down[c] : 64 KB weight stages the expert kernels
+ *                       streamed for units of token class c (0: 1-8 tokens,
+ *                       1: 9-16, 2: 17-32), up and down projections -- which
+ *                       variants actually ran.
  */
 typedef struct moe_decode_stats {
   uint64_t forwards;
   uint64_t kernels_launched;
   int32_t last_kernels;
   int32_t last_token_tiles;
+  uint64_t stages_up[3];
+  uint64_t stages_down[3];
 } moe_decode_stats;
 
 /*
@@ -192,19 +210,38 @@ int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* rout
                             void* out_host, int32_t* ids_host, float* w_host,
                             int32_t batch, void* stream_main, void* stream_aux);
 
-/* Free the workspace and events; NULL is accepted.  Synchronises the device
- * work of the handle first. */
+/* Free the workspace and events; NULL is accepted.  Waits for the handle's
+ * work first, as moe_decode_get_status does. */
 int moe_decode_destroy(moe_decode_t h);
 
 /*
- * Synchronise the handle's device, read and clear its device status word.
+ * Wait for the handle's work, then read and clear its device status word.
+ * "The handle's work" is its last forward enqueued outside graph capture
+ * (an event recorded on stream_main at its end); other streams and other
+ * handles' work are not waited for.  If the last forward was captured into
+ * a CUDA graph, its replays run on streams the handle does not know, so the
+ * whole device is synchronised instead.
  * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT (a bounded device wait gave up) or
  * MOE_ERR_DEVICE_PLAN (a device consistency check failed), or MOE_ERR_CUDA.
+ * After a device-side error the next forward re-zeroes the workspace state.
  */
 int moe_decode_get_status(moe_decode_t h);
 
-/* Copy the handle's counters to *stats (host pointer). */
+/* Copy the handle's counters to *stats (host pointer).  Waits for the
+ * handle's work first (as moe_decode_get_status) to read the device-side
+ * counters. */
 int moe_decode_get_stats(moe_decode_t h, moe_decode_stats* stats);
+
+/*
+ * Bound of every device-side wait of this handle's kernels, in probes (one
+ * probe is one mbarrier try_wait, which may itself suspend for a while, or
+ * one poll of a flag in global memory); 0 restores the default (2^24, well
+ * under a minute for a wait that never ends).  A wait that runs out records
+ * MOE_ERR_DEVICE_TIMEOUT in the status word, stops its CTA's work and lets
+ * the kernel finish.  Applies to forwards enqueued after the call (a
+ * captured graph keeps the limit it was captured with).  Host only.
+ */
+int moe_decode_set_wait_limit(moe_decode_t h, uint32_t probes);
 
 /* Static string for a MOE_* code; never NULL. */
 const char* moe_decode_error_string(int code);
@@ -272,6 +309,18 @@ int moe_decode_set_timing_events(moe_decode_t h, void* const* events, int32_t n_
 int moe_router_topk_noalloc(const void* x, const void* router_w, const float* router_bias,
                             int32_t* topk_ids, float* topk_w, int32_t batch, int32_t hidden,
                             int32_t n_experts, int32_t top_k, void* stream);
+
+/*
+ * Device status of the last moe_router_topk_noalloc call on the current
+ * device: synchronises `stream` (the stream that call was made on), reads
+ * the status word in the static scratch array and clears it.  Returns
+ * MOE_OK (also when no call has run on this device), MOE_ERR_DEVICE_TIMEOUT
+ * (a bounded wait in the router kernel gave up: the ids and weights may be
+ * wrong), MOE_ERR_DEVICE_PLAN or MOE_ERR_CUDA.  It allocates nothing (a
+ * synchronous 4-byte copy); it synchronises, so it cannot be called while
+ * `stream` is being captured.
+ */
+int moe_router_topk_noalloc_status(void* stream);
 
 /* Workspace bytes that moe_decode_init would allocate for these shapes (0 if
  * the shapes are invalid).  Pure host computation. */

@@ -32,11 +32,13 @@ EXPORTED = (
     "moe_decode_init", "moe_decode_forward", "moe_decode_forward_host", "moe_decode_destroy",
     "moe_decode_get_status", "moe_decode_get_stats", "moe_decode_error_string",
     "moe_decode_last_cuda_error", "moe_decode_last_cuda_error_string", "moe_decode_workspace_bytes",
-    "moe_decode_set_timing_events", "moe_router_topk_noalloc",
+    "moe_decode_set_timing_events", "moe_decode_set_wait_limit", "moe_router_topk_noalloc",
+    "moe_router_topk_noalloc_status",
 )
 MOE_TIMING_EVENTS = 6
 MOE_FLAG_TWO_STREAM = 1
 MOE_FLAG_TCGEN05 = 2
+MOE_FLAG_TEST_HOLD_PANEL = 4
 
 
 class Shapes(ctypes.Structure):
@@ -51,6 +53,7 @@ class Stats(ctypes.Structure):
     _fields_ = [
         ("forwards", ctypes.c_uint64), ("kernels_launched", ctypes.c_uint64),
         ("last_kernels", ctypes.c_int32), ("last_token_tiles", ctypes.c_int32),
+        ("stages_up", ctypes.c_uint64 * 3), ("stages_down", ctypes.c_uint64 * 3),
     ]
 
 
@@ -102,6 +105,10 @@ def load_library() -> ctypes.CDLL:
     lib.moe_router_topk_noalloc.argtypes = [P, P, P, P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                             ctypes.c_int32, P]
     lib.moe_router_topk_noalloc.restype = I
+    lib.moe_router_topk_noalloc_status.argtypes = [P]
+    lib.moe_router_topk_noalloc_status.restype = I
+    lib.moe_decode_set_wait_limit.argtypes = [P, ctypes.c_uint32]
+    lib.moe_decode_set_wait_limit.restype = I
     lib.moe_decode_workspace_bytes.argtypes = [ctypes.POINTER(Shapes)]
     lib.moe_decode_workspace_bytes.restype = ctypes.c_uint64
     _lib = lib
@@ -143,6 +150,16 @@ def router_topk_noalloc(x, router_w, topk_ids, topk_w, top_k: int, router_bias=N
     _check(rc, "moe_router_topk_noalloc")
 
 
+def router_topk_noalloc_status(stream=None) -> int:
+    """Synchronise `stream` and return the device status of the last
+    allocation-free router call on the current device (MOE_OK or an
+    MOE_ERR_* code); the status word is cleared."""
+    import torch
+    lib = load_library()
+    sm = _stream_handle(stream if stream is not None else torch.cuda.current_stream())
+    return lib.moe_router_topk_noalloc_status(sm)
+
+
 class MoEDecode:
     """One MoE block shape bound to the current CUDA device (owns a workspace).
 
@@ -153,12 +170,12 @@ class MoEDecode:
 
     def __init__(self, hidden: int, n_experts: int, top_k: int, inter: int, shared_inter: int = 0,
                  n_shared: int = 1, max_batch: int = 64, router_bias=None, two_stream: bool = False,
-                 tcgen05: bool = False):
+                 tcgen05: bool = False, extra_flags: int = 0):
         self._lib = load_library()
         self._bias = router_bias  # keep the device tensor alive
         self.two_stream = bool(two_stream)
         self.tcgen05 = bool(tcgen05)
-        flags = (MOE_FLAG_TWO_STREAM if two_stream else 0) | (MOE_FLAG_TCGEN05 if tcgen05 else 0)
+        flags = (MOE_FLAG_TWO_STREAM if two_stream else 0) | (MOE_FLAG_TCGEN05 if tcgen05 else 0) | int(extra_flags)
         self.shapes = Shapes(hidden, n_experts, top_k, inter, shared_inter if n_shared else 0, n_shared,
                              max_batch, _ptr(router_bias), flags)
         h = ctypes.c_void_p()
@@ -241,14 +258,20 @@ class MoEDecode:
                "moe_decode_set_timing_events")
 
     def status(self) -> int:
-        """Synchronise and return the device status (MOE_OK or an MOE_ERR_* code)."""
+        """Wait for the handle's work and return the device status (MOE_OK or an
+        MOE_ERR_* code)."""
         return self._lib.moe_decode_get_status(self._h)
+
+    def set_wait_limit(self, probes: int = 0):
+        """Bound of the kernels' device-side waits in probes (0: the default)."""
+        _check(self._lib.moe_decode_set_wait_limit(self._h, int(probes)), "moe_decode_set_wait_limit")
 
     def stats(self) -> dict:
         s = Stats()
         _check(self._lib.moe_decode_get_stats(self._h, ctypes.byref(s)), "moe_decode_get_stats")
         return {"forwards": s.forwards, "kernels_launched": s.kernels_launched, "last_kernels": s.last_kernels,
-                "last_token_tiles": s.last_token_tiles}
+                "last_token_tiles": s.last_token_tiles, "stages_up": list(s.stages_up),
+                "stages_down": list(s.stages_down)}
 
     def close(self):
         if getattr(self, "_h", None):

@@ -171,6 +171,9 @@ struct MmaArgs {
   unsigned* panel_ready_s;
   unsigned* queue;           // [0] ticket counter, [1] finished CTAs (zero between calls), [2] launch epoch
   int* status;
+  unsigned long long* stage_counts;  // [kNumClasses * 2]: stages issued per (token class, UP / DOWN), cumulative
+  uint32_t spin_limit;       // probes before a bounded wait gives up
+  int hold_panel;            // testing only: routed UP panel whose publication is withheld (-1: none)
 };
 
 // Producer's copy of the plan in shared memory: per unit the expert id,
@@ -412,7 +415,9 @@ struct SmemView {
   uint64_t* full;
   uint64_t* empty;
   StageHdr* hdr;
-  volatile int* s_misc;  // [0]: abort flag (a bounded wait gave up), [2]: stages issued
+  volatile int* s_misc;  // [0]: abort flag (a bounded wait gave up), [1]: wait limit (probes),
+                         // [2]: stages issued,
+                         // [4 + 2 * cls + (DOWN ? 1 : 0)]: stages issued per token class
   uint16_t* s_uexp;      // [kMaxUnits]
   uint16_t* s_ubeg;      // [kMaxUnits]
   uint16_t* s_aslot;     // [kMaxAssign]
@@ -580,7 +585,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         c_beg += S_A;
         c_end += S_A;
       }
-      if (*abort_flag) break;
+      if (warp_aborted(abort_flag)) break;
       int tk_next = 0;  // next ticket now: its latency overlaps this chunk
       if (lane == 0) tk_next = (int)atomicAdd(&args.queue[0], 1u);
       int piece_start = c_beg;
@@ -644,7 +649,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
             if (lane == 0) {
               uint32_t it = 0;
               while (ld_acquire_u32(pr) != ready_mark) {
-                if (++it > kSpinLimit || *abort_flag) {
+                if (++it > (uint32_t)s_misc[1] || *abort_flag) {
                   atomicCAS(args.status, kStatusOk, kStatusTimeout);
                   *abort_flag = 1;
                   ok = 0;
@@ -667,9 +672,9 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         }
         const int slot = q % NS;
         const uint32_t ph = (q / NS) & 1u;
-        bool go = mbar_wait_abortable(&empty[slot], ph ^ 1u, args.status, abort_flag) && !*abort_flag;
-        go = __all_sync(0xffffffffu, go);
-        if (!go) {
+        const bool free_slot =
+            mbar_wait_abortable_warp(&empty[slot], ph ^ 1u, args.status, abort_flag);
+        if (!free_slot || warp_aborted(abort_flag)) {
           stop = true;
           break;
         }
@@ -731,20 +736,27 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
             bulk_copy_g2s(sw + (size_t)r * pitch, u_W + (size_t)(row0 + r) * H + c0, wbytes, &full[slot], pol);
         }
         if (lane < ntok) bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, act, (uint32_t)nrows * 2, &full[slot]);
-        if (lane == 0) s_misc[2] = (int)(q + 1);
+        if (lane == 0) {
+          s_misc[2] = (int)(q + 1);
+          s_misc[4 + 2 * cls + (up ? 0 : 1)] += 1;
+        }
       }
       if (stop) break;
       tk = __shfl_sync(0xffffffffu, tk_next, 0);
     }
-    // tell the consumers there is no more work (after an abort they stop on
-    // their own: their waits give up once the abort flag is set)
+    // tell the consumers there is no more work.  Only into a slot the
+    // consumers have handed back: if that wait gave up, a stage may still
+    // own the slot (its header in use, its barrier's phase not complete),
+    // and an arrival there would fall outside the barrier's phase count --
+    // after an abort the consumers stop on their own, as their waits give up
+    // once the abort flag is set
     const int slot = q % NS;
     const uint32_t ph = (q / NS) & 1u;
-    mbar_wait_abortable(&empty[slot], ph ^ 1u, args.status, abort_flag);
-    if (lane == 0) {
+    if (mbar_wait_abortable_warp(&empty[slot], ph ^ 1u, args.status, abort_flag) && lane == 0) {
       hdr[slot].kind = kKindEnd;
       mbar_arrive(&full[slot]);
     }
+    __syncwarp();
 }
 
 template <int KC, bool TMAP>
@@ -769,8 +781,8 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], CW);
     }
-    s_misc[0] = 0;
-    s_misc[2] = 0;
+    for (int i = 0; i < 16; ++i) s_misc[i] = 0;
+    s_misc[1] = (int)min(args.spin_limit, 0x7fffffffu);
     mbar_fence_init();
   }
   __syncthreads();
@@ -793,11 +805,13 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
     while (true) {
       const int slot = q % NS;
       const uint32_t ph = (q / NS) & 1u;
-      const bool landed = mbar_wait_abortable(&full[slot], ph, args.status, abort_flag);
+      // (warp-uniform: the stage's ldmatrix / mma.sync need all 32 lanes)
+      const bool landed = mbar_wait_abortable_warp(&full[slot], ph, args.status, abort_flag);
+      if (!landed) break;
       // the header stays valid until this warp releases the slot (below,
       // once the stage's tensor-core work is done)
       const StageHdr& hd = hdr[slot];
-      if (!landed || hd.kind == kKindEnd) break;
+      if (__shfl_sync(0xffffffffu, hd.kind, 0) == kKindEnd) break;
       const bool up = hd.kind == kKindUp;
       const bool sh = hd.seg == 0;
       const int Iu = sh ? args.Is : args.I;
@@ -839,7 +853,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
         // ------------------------------------------- flush the piece's sums
         float* fbase = up ? (sh ? args.h_s : args.h) : args.acc;
         const size_t ld = up ? 2 * (size_t)Iu : (size_t)H;
-        if (!*abort_flag) {
+        if (!warp_aborted(abort_flag)) {
           if (cls == 0)
             flush_piece<0, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
           else if constexpr (KC >= 1) {
@@ -895,7 +909,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
             __syncwarp();
             if (lane == 0) {
               pcnt[panel] = 0u;
-              atomicExch(&pready[panel], ready_mark);  // publish after the fence above
+              if (sh || panel != args.hold_panel) atomicExch(&pready[panel], ready_mark);  // publish after the fence
             }
           }
         }
@@ -906,11 +920,17 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   // ------------------------------------------------------------------ exit
   __syncthreads();
   if (*abort_flag && tid == 0) {
+    // copies still in flight land in this CTA's shared memory: wait for the
+    // last NS stages issued (the ring holds no more) before the CTA exits,
+    // with the default limit (a copy in flight always lands; the runtime
+    // limit may be short)
     const int issued = s_misc[2];
     for (int qq = max(0, issued - NS); qq < issued; ++qq)
       mbar_wait_bounded(&full[qq % NS], (uint32_t)(qq / NS) & 1u, args.status);
   }
   if (tid == 0) {
+    for (int i = 0; i < 2 * kNumClasses; ++i)
+      if (s_misc[4 + i]) atomicAdd(&args.stage_counts[i], (unsigned long long)s_misc[4 + i]);
     // the last CTA out returns the counters to zero and advances the epoch
     __threadfence();
     const unsigned done = atomicAdd(&args.queue[1], 1u);

@@ -138,8 +138,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&acc_empty[b], 4);
     }
     mbar_init(mma_done, 1);
-    s_misc[0] = 0;
-    s_misc[2] = 0;
+    for (int i = 0; i < 16; ++i) s_misc[i] = 0;
+    s_misc[1] = (int)min(args.spin_limit, 0x7fffffffu);
     mbar_fence_init();
   }
   if (warp == 1) {
@@ -161,22 +161,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ================================================================= MMA
     uint32_t q = 0, piece = 0;
-    while (true) {
-      const int slot = q % NS;
-      const uint32_t ph = (q / NS) & 1u;
-      const bool landed = mbar_wait_abortable(&full[slot], ph, args.status, abort_flag);
-      const StageHdr& hd = hdr[slot];
-      const int b = piece & 1;
-      if (!landed || hd.kind == kKindEnd) {
-        // tell the epilogue warps there is no more work -- once they are done
-        // with the descriptor of the piece that last used this buffer
-        mbar_wait_abortable(&acc_empty[b], ((piece >> 1) & 1u) ^ 1u, args.status, abort_flag);
+    // Tell the epilogue warps there is no more work -- once they are done
+    // with the descriptor of the piece that last used buffer b.  If that wait
+    // gives up, nothing is posted (the buffer's barrier may still have a
+    // phase in flight, and its descriptor may be in use): the epilogue warps
+    // stop on the abort flag instead.
+    auto post_end = [&](int b) {
+      if (mbar_wait_abortable_warp(&acc_empty[b], ((piece >> 1) & 1u) ^ 1u, args.status, abort_flag)) {
         if (lane == 0) pdesc[b].kind = kKindEnd;
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&acc_full[b]);
           mbar_arrive(&acc_full[b]);
         }
+      }
+      __syncwarp();
+    };
+    while (true) {
+      const int slot = q % NS;
+      const uint32_t ph = (q / NS) & 1u;
+      // (warp-uniform: everything below is warp-collective)
+      const bool landed = mbar_wait_abortable_warp(&full[slot], ph, args.status, abort_flag);
+      const int b = piece & 1;
+      if (!landed) {
+        post_end(b);
+        break;
+      }
+      const StageHdr& hd = hdr[slot];
+      if (__shfl_sync(0xffffffffu, hd.kind, 0) == kKindEnd) {
+        post_end(b);
         break;
       }
       const bool up = hd.kind == kKindUp;
@@ -195,27 +208,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *abort_flag = 1;
         }
         __syncwarp();
-        mbar_wait_abortable(&acc_empty[b], ((piece >> 1) & 1u) ^ 1u, args.status, abort_flag);
-        if (lane == 0) pdesc[b].kind = kKindEnd;
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&acc_full[b]);
-          mbar_arrive(&acc_full[b]);
-        }
+        post_end(b);
         break;
       }
       if (flags & kFirst) {
         // the accumulator buffer must have been drained by the epilogue
         const uint32_t use = piece >> 1;
-        if (!mbar_wait_abortable(&acc_empty[b], (use & 1u) ^ 1u, args.status, abort_flag)) {
-          if (lane == 0) pdesc[b].kind = kKindEnd;
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&acc_full[b]);
-            mbar_arrive(&acc_full[b]);
-          }
-          break;
-        }
+        if (!mbar_wait_abortable_warp(&acc_empty[b], (use & 1u) ^ 1u, args.status, abort_flag))
+          break;  // the abort flag is set: the epilogue warps stop on it
         tc_fence_after();
       }
       // B operand: the stage's token rows (x or a) in the canonical K-major
@@ -302,10 +302,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     while (true) {
       const int b = piece & 1;
       const uint32_t use = piece >> 1;
-      const bool ok = mbar_wait_abortable(&acc_full[b], use & 1u, args.status, abort_flag);
+      // (warp-uniform: tcgen05.ld below is .sync.aligned)
+      const bool ok = mbar_wait_abortable_warp(&acc_full[b], use & 1u, args.status, abort_flag);
       tc_fence_after();
+      if (!ok) break;
       const StageHdr& pd = pdesc[b];
-      if (!ok || pd.kind == kKindEnd) break;
+      if (__shfl_sync(0xffffffffu, pd.kind, 0) == kKindEnd) break;
       const bool up = pd.kind == kKindUp;
       const bool sh = pd.seg == 0;
       const int Iu = sh ? args.Is : args.I;
@@ -339,7 +341,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
-        if (*abort_flag) continue;
+        if (warp_aborted(abort_flag)) continue;
         // column cc + i holds token (cc + i) % N of 128-column block (cc + i) / N
         for (int t = 0; t < N && t < ntok; ++t) {
           const int r = __shfl_sync(0xffffffffu, my_row, t);
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       ++piece;
-      if (up && !*abort_flag) {
+      if (up && !warp_aborted(abort_flag)) {
         // ---------------- last warp to finish a panel applies the SwiGLU
         __threadfence();
         __syncwarp();
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           __syncwarp();
           if (lane == 0) {
             pcnt[panel] = 0u;
-            atomicExch(&pready[panel], ready_mark);  // publish after the fence above
+            if (sh || panel != args.hold_panel) atomicExch(&pready[panel], ready_mark);  // publish after the fence
           }
         }
       }
@@ -412,11 +414,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
   if (*abort_flag && tid == 0) {
+    // copies still in flight land in this CTA's shared memory (default limit)
     const int issued = s_misc[2];
     for (int qq = max(0, issued - NS); qq < issued; ++qq)
       mbar_wait_bounded(&full[qq % NS], (uint32_t)(qq / NS) & 1u, args.status);
   }
   if (tid == 0) {
+    for (int i = 0; i < 2 * kNumClasses; ++i)
+      if (s_misc[4 + i]) atomicAdd(&args.stage_counts[i], (unsigned long long)s_misc[4 + i]);
     __threadfence();
     const unsigned done = atomicAdd(&args.queue[1], 1u);
     if (done == gridDim.x - 1) {

@@ -43,9 +43,13 @@ using moe::RouterArgs;
 
 thread_local int g_last_cuda_error = 0;
 
+// Workspace: [0, state_end) is the per-forward state (returned to zero by
+// every forward, re-zeroed after a failure); the tensor maps and the
+// device-side stage counters follow, outside that range, so re-zeroing the
+// state never destroys them.
 struct WorkspaceLayout {
   size_t status, ticket, router_epoch, logits, plan, h, a, panel_cnt, panel_ready, queue, h_s, a_s, panel_cnt_s, panel_ready_s,
-      queue_s, acc, x_stage, out_stage, ids_stage, w_stage, maps, total;
+      queue_s, acc, x_stage, out_stage, ids_stage, w_stage, state_end, maps, stage_counts, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -61,7 +65,7 @@ bool shapes_valid(const moe_decode_shapes* s) {
   if (s->n_shared != 0 && s->n_shared != 1) return false;
   if (s->n_shared == 1 && (!in(s->shared_inter, 8, 16384) || s->shared_inter % 8)) return false;
   if (!in(s->max_batch, 1, moe::kMaxBatch)) return false;
-  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05)) != 0) return false;
+  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05 | MOE_FLAG_TEST_HOLD_PANEL)) != 0) return false;
   return true;
 }
 
@@ -112,7 +116,9 @@ WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   L.out_stage = take(B * H * 2);
   L.ids_stage = take(B * k * 4);
   L.w_stage = take(B * k * 4);
+  L.state_end = off;
   L.maps = take((2 * E + 2) * (size_t)moe::kTensorMapBytes);  // tensor maps: w13[E], w2[E], shared w13, w2
+  L.stage_counts = take(2 * moe::kNumClasses * sizeof(unsigned long long));
   L.total = off;
   return L;
 }
@@ -232,6 +238,12 @@ struct moe_decode_ctx {
   WorkspaceLayout L{};
   uint8_t* ws = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+  // end of the last forward enqueued outside graph capture (what
+  // get_status / get_stats / destroy wait for); captured_last: the last
+  // forward was captured, so its work is on a stream the handle never sees
+  cudaEvent_t ev_done = nullptr;
+  bool done_recorded = false, captured_last = false;
+  uint32_t spin_limit = moe::kSpinLimit;
   bool dirty = false;
   moe_decode_stats stats{};
   ExpertTable* tab13 = nullptr;  // host staging of the pointer tables (kernel parameters)
@@ -354,7 +366,9 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   cudaError_t e;
   int kernels = 0;
   if (h->dirty) {
-    e = cudaMemsetAsync(h->ws, 0, h->L.total, sm);
+    // the per-forward state only: the tensor maps and the counters after it
+    // stay as they are
+    e = cudaMemsetAsync(h->ws, 0, h->L.state_end, sm);
     if (e != cudaSuccess) return fail_cuda(e);
     h->dirty = false;
   }
@@ -417,6 +431,10 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.panel_ready_s = h->at<unsigned>(h->L.panel_ready_s);
   base.queue = h->at<unsigned>(h->L.queue);
   base.status = status;
+  base.stage_counts = h->at<unsigned long long>(h->L.stage_counts);
+  base.spin_limit = h->spin_limit;
+  // testing only: the handle's first forward withholds routed UP panel 0
+  base.hold_panel = ((s.flags & MOE_FLAG_TEST_HOLD_PANEL) && h->stats.forwards == 0) ? 0 : -1;
 
   // Router + top-k + plan.
   RouterArgs ra{};
@@ -437,6 +455,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   ra.topk_ids = topk_ids;
   ra.topk_w = topk_w;
   ra.status = status;
+  ra.spin_limit = h->spin_limit;
   auto launch_router = [&]() -> cudaError_t {
     cudaError_t err = mark(0, sm);
     if (err != cudaSuccess) return err;
@@ -479,6 +498,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
       ga.n_su = n_su;
       ga.has_routed = 0;
       ga.queue = h->at<unsigned>(h->L.queue_s);
+      ga.hold_panel = -1;
       cudaError_t err = mark(4, st_sh);
       if (err != cudaSuccess) return err;
       err = launch(mlp, shared_grid(h, batch), mlp_threads, smem, st_sh, false, ga, *h->tab_none, *h->tab_none);
@@ -517,6 +537,17 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     if ((e = launch_combine(!fork)) != cudaSuccess) return bail(e);
   }
 
+  {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if ((e = cudaStreamIsCapturing(sm, &cap)) != cudaSuccess) return fail_cuda(e);
+    if (cap == cudaStreamCaptureStatusNone) {
+      if ((e = cudaEventRecord(h->ev_done, sm)) != cudaSuccess) return fail_cuda(e);
+      h->done_recorded = true;
+      h->captured_last = false;
+    } else {
+      h->captured_last = true;
+    }
+  }
   h->stats.forwards += 1;
   h->stats.kernels_launched += (uint64_t)kernels;
   h->stats.last_kernels = kernels;
@@ -563,6 +594,20 @@ struct DeviceGuard {
     if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
   }
 };
+
+// Wait until the handle's enqueued work is done: the event recorded at the
+// end of its last forward enqueued outside capture.  When the last forward
+// was captured into a graph, its replays run on streams the handle never
+// sees, so the whole device is synchronised instead.  Runs with the handle's
+// device current.
+int wait_for_handle_work(moe_decode_ctx* h) {
+  cudaError_t e = cudaSuccess;
+  if (h->captured_last)
+    e = cudaDeviceSynchronize();
+  else if (h->done_recorded)
+    e = cudaEventSynchronize(h->ev_done);
+  return e == cudaSuccess ? MOE_OK : fail_cuda(e);
+}
 
 }  // namespace
 
@@ -670,6 +715,7 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
   ra.plan = reinterpret_cast<Plan*>(d->scratch + kNoAllocPlanOff);
   ra.topk_ids = topk_ids;
   ra.topk_w = topk_w;
+  ra.spin_limit = moe::kSpinLimit;
   const size_t smem = moe::router_smem_bytes(batch, n_experts, ra.chunk_rows);
   cudaFuncAttributes fa{};
   const RouterKernel rk = pick_router(n_experts);
@@ -681,6 +727,25 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
   e = launch(rk, ra.G, router_threads_for(n_experts), smem, st, false, ra);
   if (e != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
+}
+
+int moe_router_topk_noalloc_status(void* stream) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_NO_DEVICE;
+  uint8_t* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_dev[dev].ready) scratch = g_noalloc_dev[dev].scratch;
+  }
+  if (!scratch) return MOE_OK;  // no call has run on this device
+  if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) return fail_cuda(e);
+  int st = 0;
+  if ((e = cudaMemcpy(&st, scratch, sizeof st, cudaMemcpyDeviceToHost)) != cudaSuccess) return fail_cuda(e);
+  if (st == moe::kStatusOk) return MOE_OK;
+  if ((e = cudaMemset(scratch, 0, sizeof st)) != cudaSuccess) return fail_cuda(e);
+  return st == moe::kStatusTimeout ? MOE_ERR_DEVICE_TIMEOUT : MOE_ERR_DEVICE_PLAN;
 }
 
 uint64_t moe_decode_workspace_bytes(const moe_decode_shapes* shapes) {
@@ -755,6 +820,8 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
   if (rc == MOE_OK && (e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming)) != cudaSuccess)
     rc = fail_cuda(e);
   if (rc == MOE_OK && (e = cudaEventCreateWithFlags(&h->ev_maps, cudaEventDisableTiming)) != cudaSuccess)
+    rc = fail_cuda(e);
+  if (rc == MOE_OK && (e = cudaEventCreateWithFlags(&h->ev_done, cudaEventDisableTiming)) != cudaSuccess)
     rc = fail_cuda(e);
   if (rc == MOE_OK) {
     // tensor-map path: shapes in whole 64-column chunks and a working encoder
@@ -838,10 +905,11 @@ int moe_decode_destroy(moe_decode_t h) {
   {
     DeviceGuard guard(h->device);
     if (h->ws) {
-      cudaError_t e = cudaDeviceSynchronize();
-      if (e != cudaSuccess) rc = fail_cuda(e);
+      const int wrc = wait_for_handle_work(h);
+      if (wrc != MOE_OK) rc = wrc;
       cudaFree(h->ws);
     }
+    if (h->ev_done) cudaEventDestroy(h->ev_done);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
     if (h->ev_maps) cudaEventDestroy(h->ev_maps);
@@ -857,8 +925,9 @@ int moe_decode_destroy(moe_decode_t h) {
 int moe_decode_get_status(moe_decode_t h) {
   if (!h) return MOE_ERR_INVALID_ARG;
   DeviceGuard guard(h->device);
-  cudaError_t e = cudaDeviceSynchronize();
-  if (e != cudaSuccess) return fail_cuda(e);
+  const int wrc = wait_for_handle_work(h);
+  if (wrc != MOE_OK) return wrc;
+  cudaError_t e;
   int st = 0;
   int* dst = h->at<int>(h->L.status);
   if ((e = cudaMemcpy(&st, dst, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess) return fail_cuda(e);
@@ -886,7 +955,23 @@ int moe_decode_set_timing_events(moe_decode_t h, void* const* events, int32_t n_
 
 int moe_decode_get_stats(moe_decode_t h, moe_decode_stats* stats) {
   if (!h || !stats) return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  const int wrc = wait_for_handle_work(h);
+  if (wrc != MOE_OK) return wrc;
+  unsigned long long c[2 * moe::kNumClasses] = {};
+  cudaError_t e = cudaMemcpy(c, h->ws + h->L.stage_counts, sizeof c, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_cuda(e);
   *stats = h->stats;
+  for (int i = 0; i < moe::kNumClasses; ++i) {
+    stats->stages_up[i] = c[2 * i];
+    stats->stages_down[i] = c[2 * i + 1];
+  }
+  return MOE_OK;
+}
+
+int moe_decode_set_wait_limit(moe_decode_t h, uint32_t probes) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  h->spin_limit = probes == 0 ? moe::kSpinLimit : probes;
   return MOE_OK;
 }
 

@@ -24,8 +24,9 @@ constexpr int kStatusOk = 0;
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusPlan = 2;
 
-// Bounded-wait limit: try_wait already suspends in hardware for a while per
-// probe, so this bounds a stuck wait to well under a minute.
+// Default bounded-wait limit (probes): try_wait already suspends in hardware
+// for a while per probe, so this bounds a stuck wait to well under a minute.
+// Launches take the limit they use as an argument (a handle can shorten it).
 constexpr uint32_t kSpinLimit = 1u << 24;
 
 // Routing plan: written by the last router CTA, read by the expert kernels.
@@ -84,28 +85,57 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Wait for the phase of `bar` with the given parity; gives up after
-// kSpinLimit probes, records kStatusTimeout in *status and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+// Wait for the phase of `bar` with the given parity; gives up after `limit`
+// probes, records kStatusTimeout in *status and returns false.  The result
+// is per thread.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status,
+                                                  uint32_t limit = kSpinLimit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   atomicCAS(status, kStatusOk, kStatusTimeout);
   return false;
 }
 
-// Same, for waits inside a CTA that shares an abort flag: once any thread
-// of the CTA has given up, the others stop waiting within ~1k probes, so a
-// failed copy never turns into a hang.  Callers keep executing the same
-// barrier sequence after a failure (skipping only the work).
+// Same, for waits inside a CTA that shares control words in shared memory:
+// ctl[0] is the CTA's abort flag, ctl[1] the wait limit in probes.  Once any
+// thread of the CTA has given up, the others stop waiting within ~1k probes,
+// so a failed copy never turns into a hang.  Both words are read only every
+// 1024 probes (the limit has that granularity), so the common path holds no
+// register for them.  The result is per thread: lanes of one warp can
+// disagree (one sees the phase complete, another the flag), so a warp that
+// branches on it must first agree (mbar_wait_abortable_warp).
 __device__ __forceinline__ bool mbar_wait_abortable(uint64_t* bar, uint32_t parity, int* status,
-                                                    volatile int* abort_flag) {
+                                                    volatile int* ctl) {
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023u) == 1023u && *abort_flag) return false;
+    if ((i & 1023u) == 1023u) {
+      if (ctl[0]) return false;
+      if (i >= (uint32_t)ctl[1]) break;
+    }
   }
   atomicCAS(status, kStatusOk, kStatusTimeout);
-  *abort_flag = 1;
+  ctl[0] = 1;
   return false;
+}
+
+// Warp-uniform form: every lane waits (so each lane's later shared-memory
+// reads are ordered after the phase it observed), then the warp agrees --
+// true only if every lane saw the phase complete.  What follows such a wait
+// is warp-collective (ldmatrix / mma.sync / tcgen05.ld .sync.aligned,
+// shuffles, __syncwarp), and a warp-collective instruction reached by only
+// some lanes of a warp is undefined (on sm_100 it can raise an illegal
+// instruction), so every branch on a wait result or on the abort flag is
+// taken by whole warps.  Must be called by all 32 lanes.
+__device__ __forceinline__ bool mbar_wait_abortable_warp(uint64_t* bar, uint32_t parity, int* status,
+                                                         volatile int* ctl) {
+  const bool ok = mbar_wait_abortable(bar, parity, status, ctl);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// The CTA's abort flag, read once and agreed by the whole warp (all 32 lanes
+// must call it).
+__device__ __forceinline__ bool warp_aborted(volatile int* abort_flag) {
+  return __any_sync(0xffffffffu, *abort_flag != 0);
 }
 
 // L2 policy for weight streams: each weight byte is read once per forward,

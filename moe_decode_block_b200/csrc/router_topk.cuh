@@ -51,6 +51,7 @@ struct RouterArgs {
   int32_t* topk_ids;            // [B, k]
   float* topk_w;                // [B, k]
   int* status;
+  uint32_t spin_limit;          // probes before the slab wait gives up
 };
 
 // Tokens padded to a multiple of 8 (x is staged token-contiguous per row).
@@ -236,6 +237,7 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
   }
 
   uint32_t phase = 0;
+  bool copy_failed = false;  // block-uniform
   const int npairs = E / 2;
   const int bp = router_bpad(B);
   for (int r0 = h0; r0 < h1; r0 += a.chunk_rows) {
@@ -246,9 +248,14 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
       const int r = i / bp, t = i - r * bp;
       xs[i] = t < B ? __bfloat162float(a.x[(size_t)t * H + r0 + r]) : 0.f;
     }
-    mbar_wait_bounded(&bar, phase, a.status);
+    // the whole block agrees on the outcome: after a failed wait no thread
+    // reads the slab and no further copy is issued into it (the status word
+    // says the logits are incomplete; the plan below stays well formed)
+    if (!__syncthreads_and(mbar_wait_bounded(&bar, phase, a.status, a.spin_limit))) {
+      copy_failed = true;
+      break;
+    }
     phase ^= 1;
-    __syncthreads();
     // items: (expert pair, group of 8 tokens); a warp's lanes take
     // consecutive pairs of one group
     const int n_items = npairs * ((B + 7) / 8);
@@ -286,6 +293,10 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
       bulk_copy_g2s(rs, a.router_w + (size_t)r1 * E, bytes, &bar, pol);
     }
   }
+
+  // a copy whose wait gave up may still land in the slab: wait for it (with
+  // the default limit) before this CTA can exit
+  if (copy_failed && tid == 0) mbar_wait_bounded(&bar, phase, a.status);
 
   // ---- last CTA: top-k, weights, bucketing -------------------------------
   __threadfence();

@@ -119,11 +119,17 @@ class BlockWeights:
     router_bias: Optional[torch.Tensor]  # [E] float32 or None
 
 
-def make_weights(shape: BlockShape, seed: int = 0, device="cpu", routing: str = "uniform") -> BlockWeights:
+def make_weights(shape: BlockShape, seed: int = 0, device="cpu", routing: str = "uniform",
+                 router_device=None) -> BlockWeights:
     """All weights of one block, bf16 ~ N(0, 0.02), each expert from its own
-    sub-seed.  ``routing == "zipf"`` adds the Zipf log-prior bias."""
+    sub-seed.  ``routing == "zipf"`` adds the Zipf log-prior bias.
+    ``router_device``: where the router weights are drawn (default: ``device``);
+    the CPU and CUDA generators give different streams, so drawing them on
+    the CPU makes them reproducible without a GPU (the benchmark does, so
+    its inputs' top-k margins can be checked ahead of time)."""
     H, E, I, Is = shape.hidden, shape.n_experts, shape.inter, shape.shared_inter
-    router_w = _normal_bf16((H, E), WEIGHT_STD, seed_for(seed, "router_w"), device)
+    rdev = device if router_device is None else router_device
+    router_w = _normal_bf16((H, E), WEIGHT_STD, seed_for(seed, "router_w"), rdev).to(device)
     w13 = torch.empty(E, H, 2 * I, dtype=torch.bfloat16, device=device)
     w2 = torch.empty(E, I, H, dtype=torch.bfloat16, device=device)
     for e in range(E):
@@ -153,3 +159,11 @@ def zipf_log_prior(n_experts: int, seed: int = 0, device="cpu", s: float = ZIPF_
 def bf16_bits(t: torch.Tensor):
     """numpy uint16 view of a bf16 tensor's bit patterns (copied to host)."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view("uint16")
+
+
+def make_router(shape: BlockShape, seed: int = 0, routing: str = "uniform"):
+    """The router weights and bias of ``make_weights(..., router_device="cpu")``
+    alone, on the CPU: (router_w [H, E] bf16, bias [E] float32 or None)."""
+    router_w = _normal_bf16((shape.hidden, shape.n_experts), WEIGHT_STD, seed_for(seed, "router_w"), "cpu")
+    bias = zipf_log_prior(shape.n_experts, seed, "cpu") if routing == "zipf" else None
+    return router_w, bias

@@ -65,7 +65,7 @@ def test_workspace_bytes_and_shape_validation(lib):
     assert 0 < tiny < full
     bad = [dict(hidden=7170), dict(hidden=0), dict(n_experts=12), dict(n_experts=2048), dict(top_k=0),
            dict(top_k=33), dict(top_k=9, n_experts=8), dict(inter=100), dict(n_shared=2),
-           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=4), dict(flags=5)]
+           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=8), dict(flags=9), dict(flags=1 << 31)]
     for kw in bad:
         sh = _shapes(**kw)
         assert lib.moe_decode_workspace_bytes(ctypes.byref(sh)) == 0, kw
@@ -76,6 +76,9 @@ def test_workspace_bytes_and_shape_validation(lib):
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TWO_STREAM))) == full
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TCGEN05))) == full
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=3))) == full
+    # the testing-only hold flag is accepted too (the handle's first forward
+    # withholds one panel publication)
+    assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TEST_HOLD_PANEL))) == full
     # shared_inter is ignored when there is no shared expert
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(n_shared=0, shared_inter=0))) > 0
 
@@ -89,6 +92,7 @@ def test_null_arguments_are_rejected_on_the_host(lib):
     assert lib.moe_decode_get_stats(None, None) == mdb.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_forward(None, *([None] * 9), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_forward_host(None, *([None] * 9), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_set_wait_limit(None, 100) == mdb.MOE_ERR_INVALID_ARG
 
 
 def test_init_without_a_gpu_reports_no_device(lib):
