@@ -15,12 +15,15 @@
  *   6. out = x + sum_j w_j y_j + shared, rounded once to bf16.
  *
  * Two execution plans (chosen per handle by moe_decode_shapes.flags):
- *   default: three kernels on stream_main.  The router kernel (steps 1-2);
- *     one persistent expert kernel that streams the shared expert's up
- *     projection first -- it needs nothing from the router, so it runs while
- *     the router is still working (programmatic dependent launch) -- then the
- *     routed experts and the shared expert's down projection; the combine
- *     (step 6).  stream_aux is not used.
+ *   default: two kernels on stream_main.  The router kernel (steps 1-2, and
+ *     an L2 prefetch of the first routed weights once the selection is
+ *     known); one persistent expert kernel that streams the shared expert's
+ *     up projection first -- it needs nothing from the router, so it runs
+ *     while the router is still working (programmatic dependent launch) --
+ *     then the routed experts and the shared expert's down projection, and
+ *     finishes with the combine (step 6): the CTA that completes a block of
+ *     output columns writes it.  stream_aux is not used.  (With
+ *     MOE_FLAG_TCGEN05 the combine is a third kernel.)
  *   MOE_FLAG_TWO_STREAM: the pages' layout.  Router and routed experts on
  *     stream_main, the shared expert on stream_aux (forked and joined with
  *     events), then a separate combine kernel.
@@ -126,8 +129,8 @@ typedef struct moe_decode_ctx* moe_decode_t;
  *   forwards          : successful forwards enqueued by this handle
  *   kernels_launched  : kernels enqueued by this handle since creation
  *   last_kernels      : kernels enqueued by the last forward (default plan:
- *                       3; MOE_FLAG_TWO_STREAM: 4, or 3 without a shared
- *                       expert)
+ *                       2, 3 with MOE_FLAG_TCGEN05; MOE_FLAG_TWO_STREAM:
+ *                       4, or 3 without a shared expert)
  *   last_token_tiles  : token tiles of 8 the expert kernels were prepared for
  *                       in the last forward (ceil(min(batch, 32) / 8))
  * Device side (counted by the expert kernels as they run, cumulative since
@@ -262,7 +265,8 @@ const char* moe_decode_last_cuda_error_string(void);
  *   [4] before the shared expert, [5] after it;
  * with the default plan (all on stream_main) [0] before the router, [1] and
  * [4] after it, [2] and [5] after the expert kernel (shared + routed
- * experts), [3] after the combine.  cudaEventElapsedTime gives each kernel's duration.  Recording an event
+ * experts, and the combine, which it finishes with), [3] after the combine
+ * (right after [2] unless MOE_FLAG_TCGEN05 runs it as its own kernel).  cudaEventElapsedTime gives each kernel's duration.  Recording an event
  * between two kernels also makes the second wait for the first to finish
  * (no early launch), so timed forwards can be slightly slower.  The handle
  * keeps the array's values (not the pointer); the caller keeps the events

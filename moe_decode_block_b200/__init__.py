@@ -163,8 +163,9 @@ def router_topk_noalloc_status(stream=None) -> int:
 class MoEDecode:
     """One MoE block shape bound to the current CUDA device (owns a workspace).
 
-    two_stream=False (default): router kernel, one expert kernel (shared
-    and routed experts) and the combine on the main stream.  two_stream=True:
+    two_stream=False (default): router kernel and one expert kernel (shared
+    and routed experts, ending with the combine + residual) on the main
+    stream.  two_stream=True:
     MOE_FLAG_TWO_STREAM, the shared expert on the aux stream.  tcgen05=True:
     MOE_FLAG_TCGEN05, the expert kernel on tcgen05 with TMEM accumulators."""
 

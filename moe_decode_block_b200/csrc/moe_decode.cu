@@ -4,11 +4,14 @@
 // "Recovering time between operators": the shared expert overlaps routing,
 // weights are fetched before their consumer starts, the residual add is
 // fused into the producing epilogue, fewer launches per layer):
-//   default (three kernels, stream_main only):
-//     router+top-k+plan; the persistent expert kernel, which streams the
-//     shared expert's up projection before its grid-dependency wait (so it
-//     overlaps the router) and then the routed experts and the shared
-//     expert's down projection; combine + residual.
+//   default (two kernels, stream_main only):
+//     router+top-k+plan (+ L2 prefetch of the first routed stages); the
+//     persistent expert kernel, which streams the shared expert's up
+//     projection before its grid-dependency wait (so it overlaps the router),
+//     then the routed experts and the shared expert's down projection, and
+//     ends with the combine + residual (the CTA that completes an output
+//     column block writes it).  With MOE_FLAG_TCGEN05 the combine is a third
+//     kernel.
 //   MOE_FLAG_TWO_STREAM (four kernels, the pages' layout):
 //     stream_main: router, routed experts, [join] combine
 //     stream_aux : shared expert, forked with an event after the router
@@ -19,6 +22,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -49,7 +53,7 @@ thread_local int g_last_cuda_error = 0;
 // state never destroys them.
 struct WorkspaceLayout {
   size_t status, ticket, router_epoch, logits, plan, h, a, panel_cnt, panel_ready, queue, h_s, a_s, panel_cnt_s, panel_ready_s,
-      queue_s, acc, x_stage, out_stage, ids_stage, w_stage, state_end, maps, stage_counts, total;
+      queue_s, acc, cb_cnt, x_stage, out_stage, ids_stage, w_stage, state_end, maps, stage_counts, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -112,6 +116,7 @@ WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   L.panel_ready_s = take(su * ncp_s * 4 + 4);
   L.queue_s = take(4 * 4);
   L.acc = take(B * H * 4);
+  L.cb_cnt = take(moe::kMaxColBlocks * sizeof(unsigned));
   L.x_stage = take(B * H * 2);
   L.out_stage = take(B * H * 2);
   L.ids_stage = take(B * k * 4);
@@ -235,6 +240,8 @@ struct moe_decode_ctx {
   int grid_routed = 0, grid_shared = 0, grid_router_max = 0;
   bool grid_routed_auto = true;
   int router_chunk_rows = 0;
+  int prefetch_stages = 0;  // L2 prefetch by the router: stages of each first expert-kernel chunk
+  int lookahead = 0;        // expert kernel: L2 prefetch of the stage this many positions ahead
   WorkspaceLayout L{};
   uint8_t* ws = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
@@ -258,6 +265,13 @@ struct moe_decode_ctx {
   std::vector<const void*> map_ptrs;  // w13[E], w2[E], shared w13, shared w2 the maps describe
   bool maps_uploaded = false;
   cudaEvent_t ev_maps = nullptr;
+  // moe_decode_forward_host with pinned, mapped host buffers: the copy of x
+  // and the forward captured once into a graph and replayed while the
+  // arguments stay the same (host_key)
+  bool host_graph_on = true;
+  cudaGraphExec_t host_exec = nullptr;
+  std::vector<const void*> host_key;
+  int host_key_batch = -1, host_graph_kernels = 0;
 
   template <typename T>
   T* at(size_t off) const {
@@ -272,7 +286,7 @@ int router_grid(const moe_decode_ctx* h, int /*batch*/) {
 }
 
 // Router kernel holding E <= 32 * NV logits per lane during top-k.
-using RouterKernel = void (*)(RouterArgs);
+using RouterKernel = void (*)(RouterArgs, ExpertTable);
 RouterKernel pick_router(int n_experts) {
   if (n_experts <= 128) return moe::router_topk_kernel<4>;
   if (n_experts <= 256) return moe::router_topk_kernel<8>;
@@ -388,6 +402,9 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   const int n_su = shared_units(s, batch);
   const int kc = kernel_class(batch);
   const MlpKernel mlp = h->use_tc ? moe::expert_tc_kernel : pick_mlp(kc, h->use_tmap);
+  // default plan on mma.sync: the combine + residual runs inside the expert
+  // kernel (the CTA that completes an output column block writes it)
+  const bool fused_combine = !two_stream && !h->use_tc;
   const int mlp_threads = h->use_tc ? moe::kTcThreads : moe::expert_threads(kc);
   const int n_stages = h->use_tc ? h->n_stages_tc : h->n_stages;
   const size_t smem = h->use_tc ? moe::tc_smem_bytes(n_stages) : moe::mma_smem_bytes(n_stages);
@@ -432,6 +449,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.queue = h->at<unsigned>(h->L.queue);
   base.status = status;
   base.stage_counts = h->at<unsigned long long>(h->L.stage_counts);
+  base.lookahead = h->use_tmap ? h->lookahead : 0;
   base.spin_limit = h->spin_limit;
   // testing only: the handle's first forward withholds routed UP panel 0
   base.hold_panel = ((s.flags & MOE_FLAG_TEST_HOLD_PANEL) && h->stats.forwards == 0) ? 0 : -1;
@@ -456,11 +474,31 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   ra.topk_w = topk_w;
   ra.status = status;
   ra.spin_limit = h->spin_limit;
+  // the expert kernel that streams the routed units, for the router's L2
+  // prefetch of its first stages
+  {
+    const bool tw = (s.flags & MOE_FLAG_TWO_STREAM) != 0;
+    int g_exp = h->grid_routed;
+    if (tw && s.n_shared && sa != sm && h->grid_routed_auto) g_exp = h->num_sms - shared_grid(h, batch);
+    ra.prefetch_stages = h->prefetch_stages;
+    ra.expert_grid = g_exp < 1 ? 1 : g_exp;
+    ra.expert_kc = h->use_tc ? moe::kNumClasses - 1 : kc;
+    ra.inter = s.inter;
+    int sdn = 0;
+    if (!tw) {
+      for (int su = 0; su < n_su; ++su) {
+        const int n = std::min(moe::kMaxUnitTokens, batch - su * moe::kMaxUnitTokens);
+        const int c = std::min(moe::class_for_tokens(n), ra.expert_kc);
+        sdn += moe::unit_stages(c, false, s.hidden, s.shared_inter);
+      }
+    }
+    ra.shared_down_stages = sdn;
+  }
   auto launch_router = [&]() -> cudaError_t {
     cudaError_t err = mark(0, sm);
     if (err != cudaSuccess) return err;
     err = launch(pick_router(s.n_experts), ra.G, router_threads_for(s.n_experts),
-                 moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra);
+                 moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra, *h->tab13);
     if (err != cudaSuccess) return err;
     ++kernels;
     return mark(1, sm);
@@ -476,17 +514,25 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   };
 
   if (!two_stream) {
-    // -------------------------------------------- default: three kernels
+    // ------------------------- default: router + expert kernel (+ combine)
     MmaArgs ma = base;
     ma.n_su = n_su;
     ma.has_routed = 1;
+    if (fused_combine) {
+      ma.out = static_cast<__nv_bfloat16*>(out);
+      ma.cb_cnt = h->at<unsigned>(h->L.cb_cnt);
+    }
     if ((e = launch_router()) != cudaSuccess) return bail(e);
     if ((e = mark(4, sm)) != cudaSuccess) return bail(e);
     e = launch(mlp, h->grid_routed, mlp_threads, smem, sm, true, ma, *h->tab13, *h->tab2);
     if (e != cudaSuccess) return bail(e);
     ++kernels;
     if ((e = mark(2, sm)) != cudaSuccess || (e = mark(5, sm)) != cudaSuccess) return bail(e);
-    if ((e = launch_combine(true)) != cudaSuccess) return bail(e);
+    if (fused_combine) {
+      if ((e = mark(3, sm)) != cudaSuccess) return bail(e);
+    } else if ((e = launch_combine(true)) != cudaSuccess) {
+      return bail(e);
+    }
   } else {
     // ------------------------------------ MOE_FLAG_TWO_STREAM: four kernels
     // Shared expert (weight 1, all tokens): on stream_aux, forked after the
@@ -609,6 +655,97 @@ int wait_for_handle_work(moe_decode_ctx* h) {
   return e == cudaSuccess ? MOE_OK : fail_cuda(e);
 }
 
+int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, const void* const* w13,
+                    const void* const* w2, const void* shared_w13, const void* shared_w2, void* out,
+                    int32_t* topk_ids, float* topk_w, int batch, cudaStream_t sm, cudaStream_t sa);
+int refresh_maps(moe_decode_ctx* h, const void* const* w13, const void* const* w2, const void* sw13,
+                 const void* sw2, cudaStream_t sm);
+
+// moe_decode_forward_host with every host buffer pinned and mapped: [copy x
+// in; the forward, storing its results into the mapped buffers] as one CUDA
+// graph, captured on the first call and replayed while the arguments (every
+// pointer, the batch, the streams and the wait limit) stay the same -- one
+// graph launch instead of a copy and two or three kernel launches with
+// kilobytes of parameters each.  Synchronises stream_main.  Returns
+// MOE_ERR_UNSUPPORTED_SHAPE when the stream cannot be captured (for example
+// it is already being captured), and the caller then runs eagerly.
+int forward_host_graph(moe_decode_ctx* h, const void* x_host, const void* router_w, const void* const* w13,
+                       const void* const* w2, const void* sw13, const void* sw2, void* out_d, void* ids_d,
+                       void* w_d, int batch, cudaStream_t sm, cudaStream_t sa) {
+  const int E = h->s.n_experts;
+  std::vector<const void*> key;
+  key.reserve(2 * (size_t)E + 12);
+  key.insert(key.end(), {x_host, router_w, sw13, sw2, out_d, ids_d, w_d, (const void*)sm, (const void*)sa,
+                         reinterpret_cast<const void*>((uintptr_t)h->spin_limit)});
+  key.insert(key.end(), w13, w13 + E);
+  key.insert(key.end(), w2, w2 + E);
+  cudaError_t e;
+  if (h->dirty) {  // state to re-zero after a device error: not part of the graph
+    if ((e = cudaMemsetAsync(h->ws, 0, h->L.state_end, sm)) != cudaSuccess) return fail_cuda(e);
+    h->dirty = false;
+  }
+  if (!h->host_exec || batch != h->host_key_batch || key != h->host_key) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(sm, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
+      cudaGetLastError();
+      return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (h->use_tmap) {  // upload changed tensor maps eagerly, not from inside the graph
+      const int rc = refresh_maps(h, w13, w2, sw13, sw2, sm);
+      if (rc != MOE_OK) return rc;
+    }
+    if ((e = cudaStreamBeginCapture(sm, cudaStreamCaptureModeThreadLocal)) != cudaSuccess) return fail_cuda(e);
+    const size_t xb = (size_t)batch * h->s.hidden * 2;
+    int rc = MOE_OK;
+    e = cudaMemcpyAsync(h->ws + h->L.x_stage, x_host, xb, cudaMemcpyHostToDevice, sm);
+    if (e != cudaSuccess) rc = fail_cuda(e);
+    const uint64_t fw = h->stats.forwards, kl = h->stats.kernels_launched;
+    if (rc == MOE_OK)
+      rc = enqueue_forward(h, h->ws + h->L.x_stage, router_w, w13, w2, sw13, sw2, out_d,
+                           static_cast<int32_t*>(ids_d), static_cast<float*>(w_d), batch, sm, sa);
+    h->stats.forwards = fw;  // counted below, once per launch
+    h->stats.kernels_launched = kl;
+    cudaGraph_t g = nullptr;
+    e = cudaStreamEndCapture(sm, &g);
+    if (rc != MOE_OK || e != cudaSuccess) {
+      if (g) cudaGraphDestroy(g);
+      cudaGetLastError();
+      h->host_key.clear();
+      return rc != MOE_OK ? rc : fail_cuda(e);
+    }
+    if (h->host_exec) {
+      cudaGraphExecUpdateResultInfo info{};
+      if (cudaGraphExecUpdate(h->host_exec, g, &info) != cudaSuccess) {
+        cudaGetLastError();
+        cudaGraphExecDestroy(h->host_exec);
+        h->host_exec = nullptr;
+      }
+    }
+    if (!h->host_exec && (e = cudaGraphInstantiate(&h->host_exec, g, 0)) != cudaSuccess) {
+      cudaGraphDestroy(g);
+      h->host_exec = nullptr;
+      h->host_key.clear();
+      return fail_cuda(e);
+    }
+    cudaGraphDestroy(g);
+    h->host_key.swap(key);
+    h->host_key_batch = batch;
+    h->host_graph_kernels = h->stats.last_kernels;
+  }
+  if ((e = cudaGraphLaunch(h->host_exec, sm)) != cudaSuccess) {
+    h->dirty = true;
+    return fail_cuda(e);
+  }
+  if ((e = cudaEventRecord(h->ev_done, sm)) != cudaSuccess) return fail_cuda(e);
+  h->done_recorded = true;
+  h->captured_last = false;
+  h->stats.forwards += 1;
+  h->stats.kernels_launched += (uint64_t)h->host_graph_kernels;
+  h->stats.last_kernels = h->host_graph_kernels;
+  if ((e = cudaStreamSynchronize(sm)) != cudaSuccess) return fail_cuda(e);
+  return MOE_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -716,6 +853,7 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
   ra.topk_ids = topk_ids;
   ra.topk_w = topk_w;
   ra.spin_limit = moe::kSpinLimit;
+  ra.prefetch_stages = 0;  // no expert kernel follows
   const size_t smem = moe::router_smem_bytes(batch, n_experts, ra.chunk_rows);
   cudaFuncAttributes fa{};
   const RouterKernel rk = pick_router(n_experts);
@@ -724,7 +862,8 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
     e = cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail_cuda(e);
   }
-  e = launch(rk, ra.G, router_threads_for(n_experts), smem, st, false, ra);
+  static const ExpertTable no_experts{};  // not read: prefetch is off
+  e = launch(rk, ra.G, router_threads_for(n_experts), smem, st, false, ra, no_experts);
   if (e != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }
@@ -786,6 +925,9 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
   h->grid_routed_auto = h->grid_routed == 0;
   if (h->grid_routed == 0) h->grid_routed = h->num_sms;
   h->grid_shared = env_int("MOE_DECODE_GRID_SHARED", 0, 0, 8 * h->num_sms);  // 0: sized per call
+  h->prefetch_stages = env_int("MOE_DECODE_PREFETCH_STAGES", 0, 0, moe::kMaxChunk);
+  h->lookahead = env_int("MOE_DECODE_LOOKAHEAD", 0, 0, 64);
+  h->host_graph_on = env_int("MOE_DECODE_HOST_GRAPH", 1, 0, 1) == 1;
   {
     int gr = h->num_sms;
     const int cap = shapes->hidden / 8;
@@ -885,6 +1027,14 @@ int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* rout
   void* wd_m = idd_m ? host_buffer_device_view(w_host, 4) : nullptr;
   const bool direct = od_m && idd_m && wd_m;
   cudaError_t e;
+  // Graph path: everything pinned and mapped (a copy from pageable memory
+  // cannot be captured), no per-kernel timing, not testing a held panel.
+  if (direct && h->host_graph_on && !h->timing && !(h->s.flags & MOE_FLAG_TEST_HOLD_PANEL) &&
+      host_buffer_device_view(const_cast<void*>(x_host), 16)) {
+    rc = forward_host_graph(h, x_host, router_w, w13, w2, shared_w13, shared_w2, od_m, idd_m, wd_m, batch, sm,
+                            static_cast<cudaStream_t>(stream_aux));
+    if (rc != MOE_ERR_UNSUPPORTED_SHAPE) return rc;  // else: capture not possible here, run eagerly
+  }
   if ((e = cudaMemcpyAsync(xd, x_host, xb, cudaMemcpyHostToDevice, sm)) != cudaSuccess) return fail_cuda(e);
   rc = enqueue_forward(h, xd, router_w, w13, w2, shared_w13, shared_w2, direct ? od_m : od,
                        static_cast<int32_t*>(direct ? idd_m : idd), static_cast<float*>(direct ? wd_m : wd), batch,
@@ -909,6 +1059,7 @@ int moe_decode_destroy(moe_decode_t h) {
       if (wrc != MOE_OK) rc = wrc;
       cudaFree(h->ws);
     }
+    if (h->host_exec) cudaGraphExecDestroy(h->host_exec);
     if (h->ev_done) cudaEventDestroy(h->ev_done);
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);

@@ -48,6 +48,9 @@ FULL = BlockShape(hidden=7168, n_experts=384, top_k=8, inter=2048, shared_inter=
 # Same per-expert shapes as FULL with only 16 experts (1.4 GB of weights):
 # the small case used for detailed profiler captures.
 PROF = BlockShape(hidden=7168, n_experts=16, top_k=8, inter=2048, shared_inter=2048)
+# The full-size router (hidden 7168, 384 experts top-8) with narrow experts
+# (inter 64, ~1 GB of weights): the small case for profiling the router.
+RPROF = BlockShape(hidden=7168, n_experts=384, top_k=8, inter=64, shared_inter=64)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -77,6 +80,9 @@ WORKLOADS: Dict[str, Workload] = {
                         "profiling case: full-size experts, 16 of them (1.4 GB), batch 8"),
     "prof_b64": Workload("prof_b64", PROF, 64, "uniform",
                          "profiling case: full-size experts, 16 of them (1.4 GB), batch 64 (~32 tokens per expert)"),
+    **{f"rprof_b{b}": Workload(f"rprof_b{b}", RPROF, b, "uniform",
+                               f"router profiling case: hidden 7168, 384 experts top-8, inter 64 (~1 GB), batch {b}")
+       for b in (1, 64)},
 }
 
 

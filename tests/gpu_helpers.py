@@ -24,7 +24,7 @@ def margin_x(batch, hidden, wts, k, seed=0, device="cuda", min_gap=MIN_MARGIN):
     attempts = np.zeros(batch, dtype=np.int64)
     rb = synth.bf16_bits(wts.router_w)
     bias = bias_np(wts)
-    for _ in range(64):
+    for _ in range(256):
         x = synth.make_x(batch, hidden, seed=seed, attempts=attempts)
         if batch == 0:
             return x.to(device)
@@ -47,11 +47,12 @@ class Run:
                              two_stream=two_stream, tcgen05=tcgen05, extra_flags=extra_flags)
 
     def kernels_per_forward(self):
-        """Kernels one forward enqueues: router, expert kernel, combine by default;
+        """Kernels one forward enqueues: router and expert kernel (which ends
+        with the combine) by default, plus a combine kernel on tcgen05;
         router, routed experts, [shared expert], combine with two streams."""
         if self.blk.two_stream:
             return 4 if self.s.n_shared else 3
-        return 3
+        return 3 if self.blk.tcgen05 else 2
 
     def forward(self, x, stream_aux=None, w13=None, w2=None):
         B = x.shape[0]
@@ -78,11 +79,20 @@ def token_class(n):
 
 
 def unit_stages(c, up, H, I):
+    """Stages of a unit's UP or DOWN list.  UP: panels of lw/2 gate (+ up)
+    columns, r-row stages.  DOWN: full panels of lw columns, then a ragged
+    last panel (H mod lw columns) in the next class's geometry when it fits
+    that width."""
     lw, r = CLASS_LW[c], CLASS_ROWS[c]
     cdiv = lambda a, b: -(-a // b)
     if up:
         return cdiv(I, lw // 2) * cdiv(H, r)
-    return cdiv(H, lw) * cdiv(I, r)
+    full = (H // lw) * cdiv(I, r)
+    rem = H % lw
+    if rem == 0:
+        return full
+    g = c + 1 if c + 1 < len(CLASS_LW) and CLASS_LW[c + 1] >= rem else c
+    return full + cdiv(I, CLASS_ROWS[g])
 
 
 def expected_stages(shape, ids, batch):

@@ -182,6 +182,28 @@ def test_host_buffer_entry_point(tiny, kind, B):
     assert tiny.blk.status() == MOE_OK
 
 
+def test_host_buffer_entry_point_replays_follow_new_inputs(tiny):
+    # with pinned, mapped buffers the host-buffer entry point captures the
+    # copy of x and the forward once and replays them: new contents of the
+    # same buffers must give new results, and another batch a new capture
+    wts = tiny.wts
+    B = 6
+    x = torch.empty(B, synth.TINY.hidden, dtype=torch.bfloat16).pin_memory()
+    out = torch.empty_like(x).pin_memory()
+    ids = torch.empty(B, 2, dtype=torch.int32).pin_memory()
+    w = torch.empty(B, 2, dtype=torch.float32).pin_memory()
+    before = tiny.blk.stats()["forwards"]
+    for seed, b in ((30, B), (31, B), (32, B), (33, 4), (34, B)):
+        x[:b].copy_(margin_x(b, synth.TINY.hidden, wts, 2, seed=seed).cpu())
+        out.fill_(float("nan"))
+        ids.fill_(-1)
+        tiny.blk.forward_host(x[:b], wts.router_w, wts.w13, wts.w2, wts.shared_w13, wts.shared_w2, out[:b], ids[:b],
+                              w[:b], batch=b)
+        oracle_check(wts, 2, x[:b], out[:b], ids[:b], w[:b])
+    assert tiny.blk.stats()["forwards"] == before + 5
+    assert tiny.blk.status() == MOE_OK
+
+
 def _graph_alternating(run, xa, xb, replays=20):
     """Capture [x <- xa; forward; x <- xb; forward] in one graph and replay it:
     an activation read hoisted above a grid-dependency wait would show up as

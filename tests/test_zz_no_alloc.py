@@ -59,8 +59,10 @@ def _status(lib):
     return lib.moe_router_topk_noalloc_status(torch.cuda.current_stream().cuda_stream)
 
 
+# 1,024 experts (the scratch's limit) at batch 64; hidden 2048 spreads the
+# logits (std ~0.9) enough that rows with every top-33 gap >= 1e-3 are common
 WIDE_8 = synth.BlockShape(hidden=256, n_experts=1024, top_k=8, inter=64, shared_inter=64)
-WIDE_32 = synth.BlockShape(hidden=256, n_experts=1024, top_k=32, inter=64, shared_inter=64)
+WIDE_32 = synth.BlockShape(hidden=2048, n_experts=1024, top_k=32, inter=64, shared_inter=64)
 
 
 @pytest.mark.parametrize("shape,routing,batches", [
