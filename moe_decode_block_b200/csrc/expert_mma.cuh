@@ -133,11 +133,8 @@ enum : int { kFirst = 1, kLast = 2 };
 // Stage header, written by the producer before it arms the stage's barrier.
 // row[n]: UP -> the h row of token n of the unit; DOWN -> the output row
 // (token).  wt[n]: DOWN weight.  seg: 0 shared expert, 1 routed.
-// cls: the stage's panel geometry (class_lw / class_rows of it; the unit's
-// token class, except for a DOWN list's narrower last panel); c0: first
-// column of the panel (UP: of each half).
 struct StageHdr {
-  int kind, seg, unit, cls, cp, row0, nrows, flags, ntok, pstages, c0, pad_;  // pstages: stages of the piece (on its last)
+  int kind, seg, unit, cls, cp, row0, nrows, flags, ntok, pstages, pad_[2];  // pstages: stages of the piece (on its last)
   int row[kUnitTok];
   float wt[kUnitTok];
 };
@@ -177,11 +174,6 @@ struct MmaArgs {
   unsigned long long* stage_counts;  // [kNumClasses * 2]: stages issued per (token class, UP / DOWN), cumulative
   uint32_t spin_limit;       // probes before a bounded wait gives up
   int hold_panel;            // testing only: routed UP panel whose publication is withheld (-1: none)
-  // Fused combine (out != nullptr): the CTA that completes an output column
-  // block writes out = bf16(x + acc) for it (see fused_combine).
-  __nv_bfloat16* out;        // [B, H] bf16
-  unsigned* cb_cnt;          // [kMaxColBlocks] DOWN stages flushed per column block, zero between calls
-  int lookahead;             // tensor-map path: L2 prefetch of the stage this many positions ahead (0: none)
 };
 
 // Producer's copy of the plan in shared memory: per unit the expert id,
@@ -192,21 +184,10 @@ constexpr int kMaxSharedUnits = kMaxBatch / kUnitTok;
 constexpr int kPlanCacheBytes =
     (kMaxUnits * (2 + 2 + 1) + kMaxAssign * 2 + 3) / 4 * 4 + (kMaxUnits + kMaxSharedUnits) * 4;
 
-// Control words of an expert-kernel CTA in shared memory (SmemView::s_misc):
-// [0] abort flag, [1] wait limit, [2] stages issued, [3] routed units of the
-// plan, [4, 10) stages per class and kind, [16, 24) / [24, 32) the
-// producer's two ticket schedules (kept here, read once per chunk, rather
-// than in 16 registers), [32, 64) DOWN stages this CTA issued per output
-// column block, [64, 96) column blocks this CTA completes (fused combine).
-constexpr int kMiscInts = 96;
-// Output column blocks of the fused combine: 512 columns each.
-constexpr int kColBlock = 512;
-constexpr int kMaxColBlocks = 32;  // hidden <= 16384
-
 __host__ __device__ inline size_t mma_smem_bytes(int n_stages) {
   // + 1 KB so the ring can start on a 1024-byte boundary (128-byte swizzle)
   return 1024 + (size_t)n_stages * kStageBytesMma + 2 * kMaxStagesMma * sizeof(uint64_t) +
-         kMaxStagesMma * sizeof(StageHdr) + kMiscInts * sizeof(int) + kPlanCacheBytes;
+         kMaxStagesMma * sizeof(StageHdr) + 16 * sizeof(int) + kPlanCacheBytes;
 }
 
 // Panels and stages per panel of one unit with class `cls`, UP or DOWN list
@@ -219,29 +200,8 @@ __host__ __device__ __forceinline__ int unit_panel_stages(int cls, bool up, int 
   const int r = class_rows(cls);
   return up ? (H + r - 1) / r : (I + r - 1) / r;
 }
-// Down projection of a unit of class c: panels of class c's width lw (R-row
-// stages).  When H is not a multiple of lw and the last panel (H mod lw
-// columns) fits the next class's width lw / 2, it takes that geometry --
-// lw / 2 columns, 2R-row stages -- so its stages too hold 64 KB of weights
-// rather than (H mod lw) / lw of that.
-// (At hidden 7168, class 0 leaves a 1024-column last panel: 1024 x 32
-// stages instead of half-filled 2048 x 16 ones.)  The stage's rows still lie
-// in one UP panel of the unit (class_rows(g) divides lw / 2).
-__host__ __device__ __forceinline__ int down_full_panels(int cls, int H) { return H / class_lw(cls); }
-__host__ __device__ __forceinline__ int down_last_geo(int cls, int H) {
-  const int rem = H % class_lw(cls);
-  // at most one class narrower, so an instance compiled for token classes
-  // <= KC needs the geometries <= KC + 1 only
-  return (rem && cls + 1 < kNumClasses && class_lw(cls + 1) >= rem) ? cls + 1 : cls;
-}
-__host__ __device__ __forceinline__ int down_stages(int cls, int H, int I) {
-  const int full = down_full_panels(cls, H) * ((I + class_rows(cls) - 1) / class_rows(cls));
-  if (H % class_lw(cls) == 0) return full;
-  const int g = down_last_geo(cls, H);
-  return full + (I + class_rows(g) - 1) / class_rows(g);
-}
 __host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int I) {
-  return up ? unit_panels(cls, true, H, I) * unit_panel_stages(cls, true, H, I) : down_stages(cls, H, I);
+  return unit_panels(cls, up, H, I) * unit_panel_stages(cls, up, H, I);
 }
 
 // Ticket schedule over a segment of T stages for a grid of G CTAs
@@ -473,7 +433,7 @@ __device__ __forceinline__ SmemView carve_smem(uint8_t* raw, int NS) {
   v.empty = v.full + kMaxStagesMma;
   v.hdr = reinterpret_cast<StageHdr*>(v.empty + kMaxStagesMma);
   v.s_misc = reinterpret_cast<volatile int*>(v.hdr + kMaxStagesMma);
-  v.s_uexp = reinterpret_cast<uint16_t*>(const_cast<int*>(v.s_misc) + kMiscInts);
+  v.s_uexp = reinterpret_cast<uint16_t*>(const_cast<int*>(v.s_misc) + 16);
   v.s_ubeg = v.s_uexp + kMaxUnits;
   v.s_aslot = v.s_ubeg + kMaxUnits;
   v.s_ucnt = reinterpret_cast<uint8_t*>(v.s_aslot + kMaxAssign);
@@ -524,16 +484,9 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
       S_dn += unit_stages(c, false, H, args.Is);
     }
     const int S_A = S_up;  // segment A: the shared UP stages
-    // the two schedules live in shared memory (written by lane 0 only)
-    Sched* sch_A = reinterpret_cast<Sched*>(const_cast<int*>(s_misc) + 16);
-    Sched* sch_B = sch_A + 1;
-    static_assert(sizeof(Sched) == 8 * sizeof(int), "two schedules fill s_misc[16, 32)");
-    if (lane == 0) {
-      *sch_A = make_round(S_up, G);
-      // segment B: the routed units, read from the plan once a ticket reaches it
-      *sch_B = make_sched(S_dn, G, 4);
-    }
-    __syncwarp();
+    const Sched sch_A = make_round(S_up, G);
+    // segment B: the routed units, read from the plan once a ticket reaches it
+    Sched sch_B = make_sched(S_dn, G, 4);
     bool b_known = !args.has_routed;
     int n_units_r = 0;
     auto know_b = [&]() {
@@ -545,7 +498,6 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         n = 0;
       }
       n_units_r = n;
-      if (lane == 0) s_misc[3] = n;
       // copy the plan to shared memory, sanitised: an entry the router never
       // produces is flagged and replaced by one that keeps every access in
       // bounds
@@ -580,8 +532,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) T += __shfl_xor_sync(0xffffffffu, T, off);
       __syncwarp();
-      if (lane == 0) *sch_B = make_sched(T + S_dn, G, 4);
-      __syncwarp();
+      sch_B = make_sched(T + S_dn, G, 4);
       b_known = true;
     };
     // Cursor over the work list: group (0 shared UP, 1 routed UP, 2 shared
@@ -616,8 +567,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
     // the SM, L1 is tiny and per-stage plan loads would go to L2 every time.
     int u_seg = -1, u_unit = -1;
     bool u_up = true;
-    int u_ntok = 0, u_cls = 0, u_lw = 0, u_S = 0, u_I = 0, u_src = 0, u_dst = 0;
-    int u_nfull = 0, u_geo = 0;  // DOWN: full-width panels, geometry of the last one
+    int u_ntok = 0, u_cls = 0, u_lw = 0, u_R = 0, u_S = 0, u_I = 0, u_src = 0, u_dst = 0;
     float u_w = 1.f;
     const __nv_bfloat16* u_W = nullptr;
     const uint8_t* u_map = nullptr;
@@ -625,13 +575,13 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
     tk = __shfl_sync(0xffffffffu, tk, 0);
     while (true) {
       int c_beg, c_end;
-      if (tk < sch_A->n_tickets) {
-        sched_range(*sch_A, tk, c_beg, c_end);
+      if (tk < sch_A.n_tickets) {
+        sched_range(sch_A, tk, c_beg, c_end);
       } else {
         if (!b_known) know_b();
-        const int tr = tk - sch_A->n_tickets;
-        if (tr >= sch_B->n_tickets) break;
-        sched_range(*sch_B, tr, c_beg, c_end);
+        const int tr = tk - sch_A.n_tickets;
+        if (tr >= sch_B.n_tickets) break;
+        sched_range(sch_B, tr, c_beg, c_end);
         c_beg += S_A;
         c_end += S_A;
       }
@@ -674,28 +624,16 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
           }
           u_cls = cls_of(u_ntok);
           u_lw = class_lw(u_cls);
+          u_R = class_rows(u_cls);
           u_S = unit_panel_stages(u_cls, up, H, u_I);
-          u_nfull = up ? 0 : down_full_panels(u_cls, H);
-          u_geo = up ? u_cls : down_last_geo(u_cls, H);
         }
-        const int ntok = u_ntok, cls = u_cls, lw = u_lw, S = u_S, Iu = u_I;
+        const int ntok = u_ntok, cls = u_cls, lw = u_lw, R = u_R, S = u_S, Iu = u_I;
         const int loc = t - cur_base;
-        // panel, stage within it and the stage's geometry (UP and full DOWN
-        // panels: the unit's class; a ragged last DOWN panel: u_geo)
-        int cp, st, geo = cls, Sp = S;
-        if (up || loc < u_nfull * S) {
-          cp = loc / S;
-          st = loc - cp * S;
-        } else {
-          cp = u_nfull;
-          st = loc - u_nfull * S;
-          geo = u_geo;
-          Sp = (Iu + class_rows(geo) - 1) / class_rows(geo);
-        }
-        const int lws = class_lw(geo), R = class_rows(geo);
+        const int cp = loc / S;
+        const int st = loc - cp * S;
         if (t == c_beg || st == 0) piece_start = t;
         const bool first = (t == piece_start);
-        const bool last = (t == c_end - 1 || st == Sp - 1);
+        const bool last = (t == c_end - 1 || st == S - 1);
         const int row0 = st * R;
         const int nrows = min(R, (up ? H : Iu) - row0);
         // DOWN reads activation rows [row0, row0 + R): wait for the UP panel
@@ -741,9 +679,9 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
           break;
         }
         const int c0 = cp * (up ? lw / 2 : lw);
-        const int w = min(up ? lw / 2 : lws, (up ? Iu : H) - c0);  // columns per half (UP) or panel (DOWN)
+        const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);  // columns per half (UP) or panel (DOWN)
         const uint32_t wbytes = (uint32_t)w * 2;
-        const uint32_t pitch = (uint32_t)lws * 2 + 16, xpitch = (uint32_t)R * 2 + 16;
+        const uint32_t pitch = (uint32_t)lw * 2 + 16, xpitch = (uint32_t)R * 2 + 16;
         // tensor-map path: loads = halves x 16-row blocks x groups of 4 chunks
         const int t_ncg = (w / kChunkCols + kBoxChunks - 1) / kBoxChunks;
         const int t_nrb = R / kBoxRows;
@@ -761,9 +699,8 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
           hd.kind = up ? kKindUp : kKindDown;
           hd.seg = seg;
           hd.unit = unit;
-          hd.cls = geo;
+          hd.cls = cls;
           hd.cp = cp;
-          hd.c0 = c0;
           hd.row0 = row0;
           hd.nrows = nrows;
           hd.flags = (first ? kFirst : 0) | (last ? kLast : 0);
@@ -778,22 +715,14 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
                              : (const void*)((seg == 0 ? args.a_s : args.a) + (size_t)u_src * Iu + row0);
         if (TMAP) {
           const int per_half = t_nrb * t_ncg;
-          const int rbstride = (lws / kChunkCols) * kChunkTile;
-          const int nch_half = (up ? lws / 2 : lws) / kChunkCols;
-          // Look ahead: the stage D positions on, when it is in the same
-          // chunk and panel (then it has the same columns, D * R rows further
-          // down), starts on its way into L2 with the same boxes, so the
-          // ring's three stages are not all the bytes this SM has in flight;
-          // its TMA loads then find the weights in L2.
-          const int D = args.lookahead;
-          const bool ahead = D > 0 && t + D < c_end && st + D < Sp;
+          const int rbstride = (lw / kChunkCols) * kChunkTile;
+          const int nch_half = (up ? lw / 2 : lw) / kChunkCols;
           for (int o = lane; o < t_nops; o += 32) {
             const int hh = o / per_half, rem = o - hh * per_half;
             const int rb = rem / t_ncg, cg = rem - rb * t_ncg;
             uint8_t* dst = sw + (size_t)rb * rbstride + (size_t)(hh * nch_half + cg * kBoxChunks) * kChunkTile;
-            const int col0 = (up ? (hh ? Iu + c0 : c0) : c0) / kChunkCols + cg * kBoxChunks;
-            tma_load_3d(dst, u_map, 0, row0 + rb * kBoxRows, col0, &full[slot], pol);
-            if (ahead) tma_prefetch_3d(u_map, 0, row0 + D * R + rb * kBoxRows, col0);
+            const int col0 = up ? (hh ? Iu + c0 : c0) : c0;
+            tma_load_3d(dst, u_map, 0, row0 + rb * kBoxRows, col0 / kChunkCols + cg * kBoxChunks, &full[slot], pol);
           }
         } else if (up) {
           for (int r = lane; r < nrows; r += 32) {
@@ -809,12 +738,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         if (lane < ntok) bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, act, (uint32_t)nrows * 2, &full[slot]);
         if (lane == 0) {
           s_misc[2] = (int)(q + 1);
-          if (last) {  // counted per piece (its stages share unit, panel and columns)
-            const int ps = t - piece_start + 1;
-            s_misc[4 + 2 * cls + (up ? 0 : 1)] += ps;
-            if (!up && args.out)  // output column blocks these DOWN stages add to
-              for (int cb = c0 / kColBlock; cb <= (c0 + w - 1) / kColBlock; ++cb) s_misc[32 + cb] += ps;
-          }
+          s_misc[4 + 2 * cls + (up ? 0 : 1)] += 1;
         }
       }
       if (stop) break;
@@ -833,105 +757,6 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
       mbar_arrive(&full[slot]);
     }
     __syncwarp();
-}
-
-// DOWN stages of a unit of class c (intermediate I) that add to output
-// column block cb: those of the DOWN panel covering it.
-__device__ __forceinline__ int down_stages_covering(int c, int cb, int H, int I) {
-  const int lw = class_lw(c);
-  const int g = (cb * kColBlock < down_full_panels(c, H) * lw) ? c : down_last_geo(c, H);
-  return (I + class_rows(g) - 1) / class_rows(g);
-}
-
-// Weighted combine + residual, fused into the expert kernel's exit (pages:
-// "Hyper Optimizing Kimi K3 in vLLM", section "Recovering time between
-// operators": residual processing fused into the producing step; dependent
-// work begins as soon as its inputs exist).  Every DOWN stage adds into a
-// whole number of 512-column output blocks.  Each CTA counted, per block,
-// the DOWN stages it issued (s_misc[32 + cb]); at exit -- after every thread
-// of the CTA fenced its reductions -- warp 0 adds those counts to the
-// block's global counter, and the CTA whose add brings a block to its total
-// (every unit's stages covering it, from the plan: the same in every CTA)
-// writes out = bf16(x + acc) for the block's columns of every token and
-// returns acc and the counter to zero.  One fence per thread and at most
-// H / 512 atomics per CTA, once per launch.  Called by all threads.
-template <int KC>
-__device__ __noinline__ void fused_combine(const MmaArgs& args, volatile int* s_misc, const uint8_t* s_ucnt) {
-  const int H = args.H, B = args.batch;
-  const int n_cb = (H + kColBlock - 1) / kColBlock;
-  const int tid = threadIdx.x, lane = tid & 31;
-  if (tid < 32) {
-    // units per token class (routed, shared), the same count in every CTA
-    auto cls_of = [&](int n) { return min(class_for_tokens(n), KC); };
-    int r0 = 0, r1 = 0, r2 = 0, q0 = 0, q1 = 0, q2 = 0;
-    const int nr = s_misc[3];
-    for (int u = lane; u < nr; u += 32) {
-      const int c = cls_of(s_ucnt[u]);
-      r0 += c == 0;
-      r1 += c == 1;
-      r2 += c == 2;
-    }
-    for (int su = lane; su < args.n_su; su += 32) {
-      const int c = cls_of(min(kUnitTok, B - su * kUnitTok));
-      q0 += c == 0;
-      q1 += c == 1;
-      q2 += c == 2;
-    }
-    r0 = __reduce_add_sync(0xffffffffu, r0);
-    r1 = __reduce_add_sync(0xffffffffu, r1);
-    r2 = __reduce_add_sync(0xffffffffu, r2);
-    q0 = __reduce_add_sync(0xffffffffu, q0);
-    q1 = __reduce_add_sync(0xffffffffu, q1);
-    q2 = __reduce_add_sync(0xffffffffu, q2);
-    for (int cb = lane; cb < n_cb; cb += 32) {
-      const int own = s_misc[32 + cb];
-      int done = 0;
-      if (own) {
-        const unsigned total =
-            (unsigned)(r0 * down_stages_covering(0, cb, H, args.I) + r1 * down_stages_covering(1, cb, H, args.I) +
-                       r2 * down_stages_covering(2, cb, H, args.I) + q0 * down_stages_covering(0, cb, H, args.Is) +
-                       q1 * down_stages_covering(1, cb, H, args.Is) + q2 * down_stages_covering(2, cb, H, args.Is));
-        const unsigned old = atomicAdd(&args.cb_cnt[cb], (unsigned)own);
-        if (old + (unsigned)own == total) {
-          done = 1;
-          args.cb_cnt[cb] = 0u;  // the last add of this launch: nobody else touches it
-        }
-      }
-      s_misc[64 + cb] = done;
-    }
-    __threadfence();  // acquire side: the other CTAs' reductions before this CTA's reads of acc
-  }
-  __syncthreads();
-#pragma unroll 1
-  for (int cb = 0; cb < n_cb; ++cb) {
-    if (!s_misc[64 + cb]) continue;
-    const int per_tok = kColBlock / 8;  // 8 columns per item
-#pragma unroll 1
-    for (int i = tid; i < B * per_tok; i += blockDim.x) {
-      const int t = i / per_tok;
-      const int c = cb * kColBlock + (i - t * per_tok) * 8;
-      if (c >= H) continue;
-      const size_t o = (size_t)t * H + c;
-      const uint4 xv = *reinterpret_cast<const uint4*>(args.x + o);
-      float4* ap = reinterpret_cast<float4*>(args.acc + o);
-      const float4 a0 = __ldcg(ap), a1 = __ldcg(ap + 1);
-      float xf[8];
-      bf16x2_to_f32(xv.x, xf[0], xf[1]);
-      bf16x2_to_f32(xv.y, xf[2], xf[3]);
-      bf16x2_to_f32(xv.z, xf[4], xf[5]);
-      bf16x2_to_f32(xv.w, xf[6], xf[7]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      uint32_t ob[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(xf[2 * j] + av[2 * j], xf[2 * j + 1] + av[2 * j + 1]);
-        ob[j] = *reinterpret_cast<const uint32_t*>(&pr);
-      }
-      *reinterpret_cast<uint4*>(args.out + o) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-      __stcg(ap, make_float4(0.f, 0.f, 0.f, 0.f));
-      __stcg(ap + 1, make_float4(0.f, 0.f, 0.f, 0.f));
-    }
-  }
 }
 
 template <int KC, bool TMAP>
@@ -956,7 +781,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], CW);
     }
-    for (int i = 0; i < kMiscInts; ++i) s_misc[i] = 0;
+    for (int i = 0; i < 16; ++i) s_misc[i] = 0;
     s_misc[1] = (int)min(args.spin_limit, 0x7fffffffu);
     mbar_fence_init();
   }
@@ -975,7 +800,6 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
     // =============================================================== consumers
     // (they read nothing the router writes: the stage headers carry it)
     constexpr int NF = acc_frags(KC);
-    constexpr int GMAX = KC + 1 < kNumClasses ? KC + 1 : kNumClasses - 1;  // panel geometries a stage can have
     float acc[NF][4];
     uint32_t q = 0;
     while (true) {
@@ -985,16 +809,14 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       const bool landed = mbar_wait_abortable_warp(&full[slot], ph, args.status, abort_flag);
       if (!landed) break;
       // the header stays valid until this warp releases the slot (below,
-      // once the stage's tensor-core work is done); every lane reads the same
-      // word, written before the phase the warp observed, so the branch is
-      // uniform
+      // once the stage's tensor-core work is done)
       const StageHdr& hd = hdr[slot];
-      if (hd.kind == kKindEnd) break;
+      if (__shfl_sync(0xffffffffu, hd.kind, 0) == kKindEnd) break;
       const bool up = hd.kind == kKindUp;
       const bool sh = hd.seg == 0;
       const int Iu = sh ? args.Is : args.I;
       const int lw = class_lw(hd.cls);
-      const int c0 = hd.c0;
+      const int c0 = hd.cp * (up ? lw / 2 : lw);
       const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);
       // local layout of the stage: UP gate [0, w), up [uoff, uoff + w); DOWN [0, w)
       const int uoff = up ? (TMAP ? lw / 2 : w) : 0;
@@ -1008,14 +830,12 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       }
       const uint32_t sw = smem_addr(stages + (size_t)slot * kStageBytesMma);
       const uint32_t sx = sw + kStageWBytes;
-      // (geometries up to GMAX: a ragged last DOWN panel may take a
-      // narrower one than the unit's token class)
       if (hd.cls == 0)
         mma_stage<0, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-      else if constexpr (GMAX >= 1) {
+      else if constexpr (KC >= 1) {
         if (hd.cls == 1)
           mma_stage<1, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-        else if constexpr (GMAX >= 2)
+        else if constexpr (KC >= 2)
           mma_stage<2, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
       }
       const bool piece_end = (hd.flags & kLast) != 0;
@@ -1036,10 +856,10 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
         if (!warp_aborted(abort_flag)) {
           if (cls == 0)
             flush_piece<0, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
-          else if constexpr (GMAX >= 1) {
+          else if constexpr (KC >= 1) {
             if (cls == 1)
               flush_piece<1, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
-            else if constexpr (GMAX >= 2)
+            else if constexpr (KC >= 2)
               flush_piece<2, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
           }
         }
@@ -1098,9 +918,6 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   }
 
   // ------------------------------------------------------------------ exit
-  // (fused combine) this thread's reductions are visible device-wide before
-  // its CTA's column-block counts move
-  if (args.out) __threadfence();
   __syncthreads();
   if (*abort_flag && tid == 0) {
     // copies still in flight land in this CTA's shared memory: wait for the
@@ -1111,15 +928,6 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
     for (int qq = max(0, issued - NS); qq < issued; ++qq)
       mbar_wait_bounded(&full[qq % NS], (uint32_t)(qq / NS) & 1u, args.status);
   }
-  // (an aborted CTA leaves its blocks incomplete: the status word says so,
-  // and the re-zeroing after it clears the counters)
-  // (the plan copy's token counts, addressed from s_misc so that no pointer
-  // stays live across the consumer loop for this)
-  if (args.out && !*abort_flag)
-    fused_combine<KC>(args, s_misc,
-                      reinterpret_cast<const uint8_t*>(reinterpret_cast<const uint16_t*>(
-                                                           const_cast<const int*>(s_misc) + kMiscInts) +
-                                                       2 * kMaxUnits + kMaxAssign));
   if (tid == 0) {
     for (int i = 0; i < 2 * kNumClasses; ++i)
       if (s_misc[4 + i]) atomicAdd(&args.stage_counts[i], (unsigned long long)s_misc[4 + i]);

@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&acc_empty[b], 4);
     }
     mbar_init(mma_done, 1);
-    for (int i = 0; i < kMiscInts; ++i) s_misc[i] = 0;
+    for (int i = 0; i < 16; ++i) s_misc[i] = 0;
     s_misc[1] = (int)min(args.spin_limit, 0x7fffffffu);
     mbar_fence_init();
   }
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int Iu = hd.seg == 0 ? args.Is : args.I;
       const int cls = hd.cls, ntok = hd.ntok, flags = hd.flags, nrows = hd.nrows;
       const int lw = class_lw(cls), R = class_rows(cls);
-      const int c0 = hd.c0;
+      const int c0 = hd.cp * (up ? lw / 2 : lw);
       const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);
       const int uoff = up ? lw / 2 : 0;
       const int N = ntok <= 16 ? 16 : 32;  // M = 128 takes N in multiples of 16
@@ -244,7 +244,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           pd.unit = hd.unit;
           pd.cls = cls;
           pd.cp = hd.cp;
-          pd.c0 = hd.c0;
           pd.row0 = hd.row0;
           pd.nrows = nrows;
           pd.flags = flags;
@@ -314,7 +313,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int Iu = sh ? args.Is : args.I;
       const int cls = pd.cls, ntok = pd.ntok, cp = pd.cp, unit = pd.unit, pstages = pd.pstages;
       const int lw = class_lw(cls);
-      const int c0 = pd.c0;
+      const int c0 = cp * (up ? lw / 2 : lw);
       const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);
       const int uoff = up ? lw / 2 : 0;
       const int N = ntok <= 16 ? 16 : 32;  // M = 128 takes N in multiples of 16

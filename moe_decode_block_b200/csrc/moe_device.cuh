@@ -178,14 +178,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int c0, 
       : "memory");
 }
 
-// Tiled bulk prefetch into L2 of the same 3-D box tma_load_3d would load
-// (no data returned to the SM, no barrier, no multicast).
-__device__ __forceinline__ void tma_prefetch_3d(const void* map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(c0), "r"(c1),
-               "r"(c2)
-               : "memory");
-}
-
 // Bulk prefetch of a global range into L2 (no data returned to the SM).
 __device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");

@@ -22,9 +22,6 @@
 //     renormalised weights, writes topk_ids/topk_w, builds the bucketed plan
 //     (experts ascending, assignments sorted by token) and returns the ticket
 //     to zero for the next call.
-//   * Once the plan is known, the last CTA also starts the routed weights the
-//     expert kernel will stream first on their way into L2 (see
-//     prefetch_first_stages) while one of its warps places the assignments.
 //   * Zeroing the logits for the next call is spread over all CTAs: with two
 //     buffers used alternately (parity of a launch counter), each CTA clears
 //     a slice of the buffer the next launch will use while it runs its GEMV.
@@ -33,7 +30,6 @@
 //     traffic: it reads the logits once and writes only the results.
 #pragma once
 
-#include "expert_mma.cuh"
 #include "moe_device.cuh"
 
 namespace moe {
@@ -56,15 +52,6 @@ struct RouterArgs {
   float* topk_w;                // [B, k]
   int* status;
   uint32_t spin_limit;          // probes before the slab wait gives up
-  // L2 prefetch of the first routed stages of the expert kernel that follows
-  // (prefetch_stages == 0: none).  The other fields describe that launch:
-  // its grid, its token-class cap, the routed intermediate size and the
-  // shared-expert DOWN stages its work list holds.
-  int prefetch_stages;          // stages of each of the first expert_grid chunks
-  int expert_grid;
-  int expert_kc;
-  int inter;
-  int shared_down_stages;
 };
 
 // Tokens padded to a multiple of 8 (x is staged token-contiguous per row).
@@ -79,8 +66,7 @@ __host__ __device__ inline int router_stage_tokens(int B, int E) {
 // Shared memory needed by router_topk_kernel for these sizes.
 __host__ __device__ inline size_t router_smem_bytes(int B, int E, int chunk_rows) {
   size_t gemv = (size_t)chunk_rows * E * 2 + (size_t)router_bpad(B) * chunk_rows * 4;
-  size_t topk = (size_t)kMaxAssign * 8 + (size_t)E * 16 + 64 + ((size_t)router_stage_tokens(B, E) + 1) * E * 4 +
-                (size_t)kMaxUnits * 4;
+  size_t topk = (size_t)kMaxAssign * 8 + (size_t)E * 16 + 64 + ((size_t)router_stage_tokens(B, E) + 1) * E * 4;
   gemv = (gemv + 15) / 16 * 16;
   return gemv > topk ? gemv : topk;
 }
@@ -206,57 +192,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 // 512-thread block leaves.
 __host__ __device__ constexpr int router_threads(int nv) { return nv <= 16 ? 512 : 256; }
 
-// L2 prefetch of the routed weights the expert kernel streams first.  Its
-// work list after the shared expert's UP stages (segment B) starts with the
-// routed UP stages, unit after unit in plan order; its first tickets hand
-// out chunks [j * c_big, (j + 1) * c_big) of that list, one per CTA, j <
-// expert_grid, and each CTA streams its chunk's stages in order.  So the
-// first P stages of each of those chunks are the weights wanted first once
-// the plan is visible; this starts them on their way into L2 (bulk
-// prefetch, nothing returns to the SM) while the plan is still being
-// finished and the expert kernel's grid-dependency wait has not returned.
-// s_units: per unit (expert << 8) | tokens; T: stages of the whole segment.
-// Called by the threads [t0, t0 + nthr) of the last CTA.
-__device__ __forceinline__ void prefetch_first_stages(const RouterArgs& a, const ExpertTable& w13,
-                                                      const uint32_t* s_units, int n_units, int T, int t0,
-                                                      int nthr) {
-  const int P = a.prefetch_stages, G = a.expert_grid, H = a.H, I = a.inter;
-  const int c_big = min(max(T / (4 * G), 1), kMaxChunk);  // make_sched's chunk for div = 4
-  if (P > c_big) return;  // chunks too short for the first P stages to belong to one chunk
-  for (int i = threadIdx.x - t0; i < G * P; i += nthr) {
-    const int t = (i / P) * c_big + i % P;  // stage of segment B
-    int base = 0, u = 0, cls = 0, S = 0;
-    for (; u < n_units; ++u) {
-      const int n = (int)(s_units[u] & 0xffu);
-      cls = min(class_for_tokens(n), a.expert_kc);
-      S = unit_stages(cls, true, H, I);
-      if (t < base + S) break;
-      base += S;
-    }
-    if (u == n_units) continue;  // past the routed UP stages
-    const int e = (int)(s_units[u] >> 8);
-    const int lw = class_lw(cls), R = class_rows(cls);
-    const int Sp = unit_panel_stages(cls, true, H, I);
-    const int loc = t - base, cp = loc / Sp, st = loc - cp * Sp;
-    (void)lw;
-    // the stage's rows as one contiguous block (both halves of every UP
-    // panel of those rows: one operation instead of two per row)
-    const int r0 = st * R, nr = min(R, H - r0);
-    bulk_prefetch_l2(w13.p[e] + (size_t)r0 * 2 * I, (uint32_t)nr * 2 * I * 2);
-    (void)cp;
-  }
-}
-
 template <int NV>
-__global__ void __launch_bounds__(router_threads(NV), 1)
-    router_topk_kernel(const __grid_constant__ RouterArgs a, const __grid_constant__ ExpertTable w13) {
+__global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(const __grid_constant__ RouterArgs a) {
   constexpr int NT = router_threads(NV);
   extern __shared__ __align__(1024) uint8_t router_smem[];
   uint8_t* smem = router_smem;
   __shared__ __align__(8) uint64_t bar;
   __shared__ int s_last;
   __shared__ int s_warp[NT / 32 + 1];
-  __shared__ int s_stages;  // stages of the expert kernel's segment B (prefetch)
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E, B = a.B, H = a.H, k = a.k;
@@ -482,12 +425,10 @@ __global__ void __launch_bounds__(router_threads(NV), 1)
     __syncthreads();  // the staging buffer is reused by the next group of tokens
   }
   for (int e = tid; e < E; e += NT) s_cnt[e] = 0;
-  if (tid == 0) s_stages = a.shared_down_stages;
   __syncthreads();
   const int nas = B * k;
   for (int i = tid; i < nas; i += NT) atomicAdd(&s_cnt[s_ids[i]], 1);
   __syncthreads();
-  uint32_t* s_units = reinterpret_cast<uint32_t*>(s_lg + (size_t)TB * E);  // [kMaxUnits]
 
   // Exclusive scans of counts and of units per expert over E (<= 1024 =
   // 4/thread); an expert with c tokens gets ceil(c / kMaxUnitTokens) units.
@@ -503,7 +444,6 @@ __global__ void __launch_bounds__(router_threads(NV), 1)
   int ctot, ftot;
   int cbase = block_exclusive_scan<NT>(csum, s_warp, ctot);
   int fbase = block_exclusive_scan<NT>(fsum, s_warp, ftot);
-  int my_stages = 0;  // expert-kernel stages of this thread's units (prefetch)
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int e = tid * 4 + i;
@@ -511,15 +451,9 @@ __global__ void __launch_bounds__(router_threads(NV), 1)
       s_off[e] = cbase;
       s_act[e] = f4[i] ? fbase : -1;
       for (int j = 0; j < f4[i]; ++j) {
-        const int n = min(kMaxUnitTokens, c4[i] - j * kMaxUnitTokens);
         a.plan->unit_expert[fbase + j] = e;
         a.plan->unit_begin[fbase + j] = cbase + j * kMaxUnitTokens;
-        a.plan->unit_count[fbase + j] = n;
-        if (a.prefetch_stages > 0 && fbase + j < kMaxUnits) {
-          s_units[fbase + j] = ((uint32_t)e << 8) | (uint32_t)n;
-          const int c = min(class_for_tokens(n), a.expert_kc);
-          my_stages += unit_stages(c, true, H, a.inter) + unit_stages(c, false, H, a.inter);
-        }
+        a.plan->unit_count[fbase + j] = min(kMaxUnitTokens, c4[i] - j * kMaxUnitTokens);
       }
     }
     cbase += c4[i];
@@ -529,7 +463,6 @@ __global__ void __launch_bounds__(router_threads(NV), 1)
     a.plan->n_active = ftot;
     if (ctot != nas) atomicCAS(a.status, kStatusOk, kStatusPlan);
   }
-  if (my_stages) atomicAdd(&s_stages, my_stages);
 
   __syncthreads();
   // Assignment (t, j) goes to offset[e] + #{t' < t : e in ids[t']}: one warp
@@ -551,8 +484,6 @@ __global__ void __launch_bounds__(router_threads(NV), 1)
       }
       __syncwarp();
     }
-  } else if (a.prefetch_stages > 0) {
-    prefetch_first_stages(a, w13, s_units, min(ftot, kMaxUnits), s_stages, 32, NT - 32);
   }
   if (tid == 0) {
     *a.ticket = 0u;

@@ -58,6 +58,10 @@ def _load():
         lib.oracle_expert_outputs.restype = I
         lib.oracle_combine.argtypes = [P, P, P, P, I, I, I, P]
         lib.oracle_combine.restype = I
+        lib.oracle_expert_outputs_fp8.argtypes = [P, I, I, P, P, P, P, I, I, P, P]
+        lib.oracle_expert_outputs_fp8.restype = I
+        lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_value.restype = ctypes.c_double
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = I
         _lib = lib
@@ -176,6 +180,53 @@ def block_streamed(x, ids, w, fetch_expert, sw13=None, sw2=None):
     s = None
     if sw13 is not None:
         s = expert_outputs(x, sw13, sw2, np.arange(B))
+    out = np.zeros((B, H), np.float64)
+    _check(lib.oracle_combine(_ptr(x), _ptr(w), _ptr(y), _ptr(s), B, H, k, _ptr(out)), "oracle_combine")
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    """The fp64 value of an 8-bit e4m3 code (NaN for the NaN codes)."""
+    return float(_load().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def expert_outputs_fp8(x, q13, s13, q2, s2, rows):
+    """Step 5 for one expert with block-scaled e4m3 weights (C oracle):
+    q13 uint8 [2I, H] with fp32 scales [ceil(2I/128), ceil(H/128)], q2 uint8
+    [H, I] with scales [ceil(H/128), ceil(I/128)]; y [len(rows), H] f64."""
+    lib = _load()
+    x = _u16(x)
+    B, H = x.shape
+    q13 = np.ascontiguousarray(q13, dtype=np.uint8)
+    q2 = np.ascontiguousarray(q2, dtype=np.uint8)
+    s13 = np.ascontiguousarray(s13, dtype=np.float32)
+    s2 = np.ascontiguousarray(s2, dtype=np.float32)
+    I = q13.shape[0] // 2
+    assert q13.shape == (2 * I, H) and q2.shape == (H, I)
+    assert s13.shape == (-(-2 * I // 128), -(-H // 128)) and s2.shape == (-(-H // 128), -(-I // 128))
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    y = np.zeros((len(rows), H), np.float64)
+    _check(lib.oracle_expert_outputs_fp8(_ptr(x), B, H, _ptr(q13), _ptr(s13), _ptr(q2), _ptr(s2), I, len(rows),
+                                         _ptr(rows), _ptr(y)), "oracle_expert_outputs_fp8")
+    return y
+
+
+def block_streamed_fp8(x, ids, w, fetch_expert, shared=None):
+    """Steps 5-7 with block-scaled e4m3 expert weights, one expert at a time:
+    ``fetch_expert(e)`` returns (q13, s13, q2, s2); ``shared`` is the shared
+    expert's (q13, s13, q2, s2) or None.  The sum of step 7 is taken in the
+    same order as ``block``."""
+    lib = _load()
+    x = _u16(x)
+    B, H = x.shape
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float64)
+    k = ids.shape[1] if ids.ndim == 2 else 0
+    y = np.zeros((B, k, H), np.float64)
+    for e in sorted(set(ids.ravel().tolist())):
+        bj = np.argwhere(ids == e)
+        y[bj[:, 0], bj[:, 1]] = expert_outputs_fp8(x, *fetch_expert(e), bj[:, 0])
+    s = None if shared is None else expert_outputs_fp8(x, *shared, np.arange(B))
     out = np.zeros((B, H), np.float64)
     _check(lib.oracle_combine(_ptr(x), _ptr(w), _ptr(y), _ptr(s), B, H, k, _ptr(out)), "oracle_combine")
     return out

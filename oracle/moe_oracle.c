@@ -216,6 +216,67 @@ done:
   return rc;
 }
 
+/* ---- FP8 expert weights (an extension the pages do not cover) ----------
+ * Weights stored as 8-bit e4m3 codes (1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits; exponent 0 is subnormal: m / 8 * 2^-6; the all-ones
+ * code is NaN, there is no infinity) in [out, in] layout, with one fp32 scale
+ * per block of 128 outputs x 128 inputs, scales row-major over
+ * [ceil(out / 128), ceil(in / 128)].  The weight of (output o, input i) is
+ * decode(q[o, i]) * scale[o / 128, i / 128], in fp64. */
+static double e4m3_to_double(uint8_t q) {
+  const int s = q >> 7, e = (q >> 3) & 15, m = q & 7;
+  if (e == 15 && m == 7) return NAN;
+  const double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+  return s ? -v : v;
+}
+
+double oracle_e4m3_value(uint8_t q) { return e4m3_to_double(q); }
+
+/* y[o] = sum_i v[i] * W[o, i] for o < nout, W the block-scaled e4m3 matrix
+ * [nout, nin] (row o contiguous); each y[o] is summed in i order by one
+ * thread. */
+static void vec_times_fp8(const double* v, const uint8_t* q, const float* sc, int nout, int nin, double* y) {
+  const int nb = (nin + 127) / 128;
+#pragma omp parallel for schedule(static)
+  for (int o = 0; o < nout; ++o) {
+    const uint8_t* row = q + (size_t)o * nin;
+    const float* srow = sc + (size_t)(o / 128) * nb;
+    double acc = 0.0;
+    for (int i = 0; i < nin; ++i) acc += v[i] * (e4m3_to_double(row[i]) * (double)srow[i / 128]);
+    y[o] = acc;
+  }
+}
+
+/* Step 5 for one expert with e4m3 weights: q13 [2I, H] (outputs 0..I-1 the
+ * gate, I..2I-1 the up projection) with scales s13, q2 [H, I] with scales
+ * s2; y[i, :] for token rows[i] of x. */
+int oracle_expert_outputs_fp8(const uint16_t* x, int B, int H, const uint8_t* q13, const float* s13,
+                              const uint8_t* q2, const float* s2, int I, int n, const int32_t* rows,
+                              double* y) {
+  if (B < 0 || H <= 0 || I <= 0 || n < 0) return ORACLE_BAD_ARG;
+  if (n == 0) return ORACLE_OK;
+  if (!x || !q13 || !s13 || !q2 || !s2 || !rows || !y) return ORACLE_BAD_ARG;
+  double* xb = (double*)malloc(sizeof(double) * (size_t)H);
+  double* gu = (double*)malloc(sizeof(double) * 2 * (size_t)I);
+  double* a = (double*)malloc(sizeof(double) * (size_t)I);
+  int rc = ORACLE_OK;
+  if (!xb || !gu || !a) {
+    rc = ORACLE_NO_MEMORY;
+    goto done;
+  }
+  for (int i = 0; i < n; ++i) {
+    const int b = rows[i];
+    if (b < 0 || b >= B) { rc = ORACLE_BAD_ARG; goto done; }
+    for (int h = 0; h < H; ++h) xb[h] = bf16_bits_to_double(x[(size_t)b * H + h]);
+    vec_times_fp8(xb, q13, s13, 2 * I, H, gu);
+    for (int c = 0; c < I; ++c) a[c] = silu(gu[c]) * gu[I + c];
+    vec_times_fp8(a, q2, s2, H, I, y + (size_t)i * H);
+  }
+done:
+  free(xb); free(gu); free(a);
+  return rc;
+}
+
 /* Step 7 from per-assignment expert outputs: out_b = x_b + sum_j w_j y[b,j]
  * (+ s_b), with y [B,k,H] and s [B,H] (NULL: no shared expert) -- the same
  * additions, in the same order, as oracle_block. */

@@ -371,3 +371,108 @@ def test_expert_outputs_is_one_swiglu_mlp_per_row():
     resid = d["x"].astype(np.uint32) << 16
     xr = resid.view(np.float32).astype(np.float64)
     np.testing.assert_allclose(y, (full - xr)[rows], rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- FP8 expert weights ---
+
+def _fp8_expert(I, H, seed, scale_lo=0.5, scale_hi=2.0):
+    g = torch.Generator().manual_seed(seed)
+    q13 = torch.randint(0, 256, (2 * I, H), generator=g, dtype=torch.uint8)
+    q2 = torch.randint(0, 256, (H, I), generator=g, dtype=torch.uint8)
+    q13[(q13 & 0x7F) == 0x7F] = 0x38  # no NaN codes (replace with 1.0)
+    q2[(q2 & 0x7F) == 0x7F] = 0x38
+    s13 = (scale_lo + (scale_hi - scale_lo) * torch.rand(-(-2 * I // 128), -(-H // 128), generator=g)) * 2 ** -9
+    s2 = (scale_lo + (scale_hi - scale_lo) * torch.rand(-(-H // 128), -(-I // 128), generator=g)) * 2 ** -9
+    return q13.numpy(), s13.numpy().astype(np.float32), q2.numpy(), s2.numpy().astype(np.float32)
+
+
+def _torch_decode(q):
+    return torch.from_numpy(np.ascontiguousarray(q)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def test_e4m3_decoding_matches_torch_for_every_code():
+    ref = _torch_decode(np.arange(256, dtype=np.uint8))
+    for code in range(256):
+        v = oracle.e4m3_value(code)
+        if np.isnan(ref[code]):
+            assert np.isnan(v), code
+        else:
+            assert v == ref[code], (code, v, ref[code])
+    assert oracle.e4m3_value(0x7E) == 448.0 and oracle.e4m3_value(0x01) == 2.0 ** -9
+
+
+def _dequant(q, s):
+    d = _torch_decode(q)
+    o, i = q.shape
+    full = np.repeat(np.repeat(s.astype(np.float64), 128, axis=0), 128, axis=1)[:o, :i]
+    return d * full
+
+
+def test_fp8_expert_with_unit_scales_is_the_bf16_expert_bitwise():
+    # e4m3 values are exact in bf16: with unit scales the fp8 expert must be
+    # the bf16 oracle's expert on the decoded (transposed) weights, bit for bit
+    H, I = 256, 192
+    q13, s13, q2, s2 = _fp8_expert(I, H, seed=1)
+    s13[:] = 1.0
+    s2[:] = 1.0
+    x = rand_block(B=3, H=H, seed=2)["x"]
+    y8 = oracle.expert_outputs_fp8(x, q13, s13, q2, s2, [0, 2, 1])
+    w13 = to_bits(_torch_decode(q13).T.astype(np.float32))
+    w2 = to_bits(_torch_decode(q2).T.astype(np.float32))
+    y16 = oracle.expert_outputs(x, w13, w2, [0, 2, 1])
+    assert np.array_equal(y8, y16)
+
+
+def test_fp8_block_scale_applies_to_its_block_only():
+    # doubling one scale equals doubling exactly that 128 x 128 block of the
+    # dequantized weights (a power-of-two scaling is exact, and the doubled
+    # values are still exact in bf16): compare with the bf16 oracle on the
+    # decoded weights with that block doubled
+    H, I = 384, 256
+    q13, s13, q2, s2 = _fp8_expert(I, H, seed=3)
+    s13[:] = 1.0
+    s2[:] = 1.0
+    x = rand_block(B=2, H=H, seed=4)["x"]
+    s13b = s13.copy()
+    s13b[1, 2] = 2.0  # outputs 128..255, inputs 256..383
+    y = oracle.expert_outputs_fp8(x, q13, s13b, q2, s2, [0, 1])
+    d13 = _torch_decode(q13)
+    d13[128:256, 256:384] *= 2.0
+    y16 = oracle.expert_outputs(x, to_bits(d13.T.astype(np.float32)), to_bits(_torch_decode(q2).T.astype(np.float32)),
+                                [0, 1])
+    assert np.array_equal(y, y16)
+
+
+def test_fp8_expert_matches_a_library_composition():
+    # torch's e4m3 decoding, numpy fp64 matmuls and scipy's logistic function
+    H, I = 256, 160
+    q13, s13, q2, s2 = _fp8_expert(I, H, seed=5)
+    x = rand_block(B=4, H=H, seed=6)["x"]
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    W13 = _dequant(q13, s13)  # [2I, H]
+    W2 = _dequant(q2, s2)     # [H, I]
+    gu = xf @ W13.T
+    a = gu[:, :I] * scipy.special.expit(gu[:, :I]) * gu[:, I:]
+    ref = a @ W2.T
+    y = oracle.expert_outputs_fp8(x, q13, s13, q2, s2, np.arange(4))
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_fp8_streamed_block_combines_like_the_block():
+    # routing, residual and shared expert around fp8 experts: the fp8 block
+    # with unit scales equals the bf16 oracle's block on the decoded weights
+    H, I, E, k = 128, 128, 6, 2
+    experts = [_fp8_expert(I, H, seed=20 + e) for e in range(E)]
+    for q13, s13, q2, s2 in experts:
+        s13[:] = 1.0
+        s2[:] = 1.0
+    shared = _fp8_expert(I, H, seed=40)
+    shared[1][:] = 1.0
+    shared[3][:] = 1.0
+    d = rand_block(B=5, H=H, E=E, k=k, seed=7)
+    _, ids, w = oracle.router(d["x"], d["router_w"], k, None)
+    out8 = oracle.block_streamed_fp8(d["x"], ids, w, lambda e: experts[e], shared)
+    tb = lambda q: to_bits(_torch_decode(q).T.astype(np.float32))
+    out16 = oracle.block(d["x"], ids, w, [tb(e[0]) for e in experts], [tb(e[2]) for e in experts],
+                         tb(shared[0]), tb(shared[2]))
+    assert np.array_equal(out8, out16)
