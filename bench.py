@@ -380,6 +380,46 @@ def check_against_oracle(wts, x, out, ids, w, k, ref=None):
             "tol": OUT_RTOL * rms, "rows": int(x.shape[0])}
 
 
+def fp8_bytes_per_step(shape, w8, ids, batch: int):
+    """Algorithmic HBM bytes of one forward with e4m3 expert weights: each
+    distinct routed expert's codes and block scales, the shared expert's,
+    the bf16 router and the activations.  Returns (bytes, distinct)."""
+    distinct = len(set(ids.reshape(-1).tolist()))
+    per = (w8.q13[0].numel() + w8.q2[0].numel()) + 4 * (w8.s13[0].numel() + w8.s2[0].numel())
+    shared = 0 if w8.shared_q13 is None else (w8.shared_q13.numel() + w8.shared_q2.numel()
+                                             + 4 * (w8.shared_s13.numel() + w8.shared_s2.numel()))
+    act = 2 * batch * shape.hidden * 2
+    return distinct * per + shared + shape.router_bytes() + act, distinct
+
+
+def check_fp8_against_oracle(shape, w8, x, out, ids, w):
+    """An e4m3-weight forward against the fp64 oracle of block-scaled e4m3
+    weights (ids exact, weights within W_ATOL, outputs within OUT_RTOL * rms)."""
+    import numpy as np
+
+    import oracle
+    from moe_decode_block_b200 import synth
+    k, H, I, Is = shape.top_k, shape.hidden, shape.inter, shape.shared_inter
+
+    def osc(s_api, outs):  # the library's [in/128, padded] scales -> the oracle's [out/128, in/128]
+        return np.ascontiguousarray(s_api.detach().cpu().numpy()[:, :-(-outs // 128)].T)
+
+    xb = synth.bf16_bits(x)
+    bias = None if w8.router_bias is None else w8.router_bias.float().cpu().numpy()
+    _, o_ids, o_w = oracle.router(xb, synth.bf16_bits(w8.router_w), k, bias)
+    fetch = lambda e: (w8.q13[e].cpu().numpy(), osc(w8.s13[e], 2 * I), w8.q2[e].cpu().numpy(), osc(w8.s2[e], H))
+    shared = (w8.shared_q13.cpu().numpy(), osc(w8.shared_s13, 2 * Is), w8.shared_q2.cpu().numpy(),
+              osc(w8.shared_s2, H))
+    o_out = oracle.block_streamed_fp8(xb, o_ids, o_w, fetch, shared)
+    g_out = out.float().cpu().numpy()
+    ids_ok = bool(np.array_equal(ids.cpu().numpy(), o_ids))
+    w_err = float(np.max(np.abs(w.cpu().numpy().astype(np.float64) - o_w)))
+    err = float(np.max(np.abs(g_out - o_out))) if np.all(np.isfinite(g_out)) else float("inf")
+    rms = float(np.sqrt(np.mean(o_out ** 2)))
+    return {"ok": ids_ok and w_err <= W_ATOL and err <= OUT_RTOL * rms, "ids_exact": ids_ok, "max_w_err": w_err,
+            "max_out_err": err, "tol": OUT_RTOL * rms, "rows": int(x.shape[0])}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -589,6 +629,54 @@ def run_ours(args):
                              else "unchecked", "clocks": cclk}
             cases.append(case)
 
+    # ---- e4m3 expert weights (block-scaled), batch 1 and 8, same router
+    fp8 = None
+    fp8_cases = []
+    if world == 1 and not args.no_configs and s == synth.FULL and not args.two_stream:
+        w8 = synth.make_fp8_weights(s, seed=args.seed, device=dev, routing=wl.routing, router_device="cpu")
+        fp8 = {"weights": "e4m3 codes [out, in] + fp32 scale per 128 x 128 block (scale = block absmax / 448), "
+                          "router bf16, activations bf16 (f16 in the products), fp32 accumulation"}
+        for name, fb in (("fp8_b1", 1), ("fp8_b8", 8)):
+            att = x_attempts(f"full_b{fb}", args.seed) if args.seed == 0 else None
+            fx = synth.make_x(fb, s.hidden, seed=args.seed, attempts=att).to(dev)
+            fblk = MoEDecode(s.hidden, s.n_experts, s.top_k, s.inter, s.shared_inter, n_shared=s.n_shared,
+                             max_batch=fb, router_bias=w8.router_bias, fp8=True)
+            fout = torch.empty_like(fx)
+            fids = torch.empty(fb, s.top_k, dtype=torch.int32, device=dev)
+            fw = torch.empty(fb, s.top_k, dtype=torch.float32, device=dev)
+            fargs8 = (fx, w8.router_w, w8.q13, w8.s13, w8.q2, w8.s2, w8.shared_q13, w8.shared_s13, w8.shared_q2,
+                      w8.shared_s2, fout, fids, fw)
+            with torch.cuda.stream(main):
+                fblk.forward_fp8(*fargs8, stream_main=main, stream_aux=aux)
+            main.synchronize()
+            fg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(fg, stream=main):
+                fblk.forward_fp8(*fargs8, stream_main=torch.cuda.current_stream(), stream_aux=aux)
+            with torch.cuda.stream(main):
+                for _ in range(20):
+                    flush()
+                    fg.replay()
+            torch.cuda.synchronize()
+            fst = [torch.cuda.Event(enable_timing=True) for _ in range(args.config_steps)]
+            fen = [torch.cuda.Event(enable_timing=True) for _ in range(args.config_steps)]
+            with torch.cuda.stream(main):
+                for i in range(args.config_steps):
+                    flush()
+                    fst[i].record(main)
+                    fg.replay()
+                    fen[i].record(main)
+            torch.cuda.synchronize()
+            fus = 1e3 * statistics.mean(a.elapsed_time(b) for a, b in zip(fst, fen))
+            fbytes, fdist = fp8_bytes_per_step(s, w8, fids.cpu().numpy(), fb)
+            fp8[name] = {"batch": fb, "distinct_experts": fdist, "bytes_per_step": fbytes,
+                         "us_per_block": round(fus, 2), "GB/s": round(fbytes / (fus * 1e-6) / 1e9, 1),
+                         "frac_of_measured_peak": round(fbytes / (fus * 1e-6) / 1e9 / peak, 4),
+                         "tokens_per_s": round(fb / (fus * 1e-6), 1), "steps": args.config_steps,
+                         "vs_bf16_us": round(ms_per_step * 1e3, 2) if fb == B else
+                         (configs.get(f"full_b{fb}", {}).get("us_per_block") if configs else None)}
+            del fg
+            fp8_cases.append((name, fblk, fx, fout, fids, fw))
+
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N == 1); its
     # last run is the oracle output the headline forward is checked against
     cpu = None
@@ -610,6 +698,9 @@ def run_ours(args):
                   wl.name: check_against_oracle(wts, x, head.out, head.ids, head.w, s.top_k, oracle_ref)}
         for case in cases:
             parity[case.wl.name] = check_against_oracle(case.wts, case.x, case.out, case.ids, case.w, s.top_k)
+        for name, fblk, fx, fout, fids, fw in fp8_cases:
+            parity[name] = check_fp8_against_oracle(s, w8, fx, fout, fids, fw)
+            fp8[name]["parity"] = "ok" if parity[name]["ok"] else "FAIL"
         parity["ok"] = all(v["ok"] for k, v in parity.items() if isinstance(v, dict))
         if configs:
             for name in configs:
@@ -627,7 +718,7 @@ def run_ours(args):
             "bytes_per_step": bstep, "distinct_experts": distinct,
             "roofline": roofline, "kernels_us": kern_us, "cpu_baseline": cpu, "e2e": e2e,
             "parity": "ok" if parity_ok and parity is not None else ("FAIL" if not parity_ok else None),
-            "parity_detail": parity, "configs": configs,
+            "parity_detail": parity, "configs": configs, "fp8": fp8,
             "gpu_launches": head.kernels_per_step * args.steps, "kernels_per_step": head.kernels_per_step,
             "clocks": clocks, "bracket_ms_incl_flush": round(bracket_ms, 2),
             "device_status": status,
@@ -635,6 +726,8 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     for case in cases:
         case.close()
+    for _, fblk, *_rest in fp8_cases:
+        fblk.close()
     head.close()
     if world > 1:
         torch.distributed.barrier()

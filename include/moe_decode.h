@@ -15,15 +15,12 @@
  *   6. out = x + sum_j w_j y_j + shared, rounded once to bf16.
  *
  * Two execution plans (chosen per handle by moe_decode_shapes.flags):
- *   default: two kernels on stream_main.  The router kernel (steps 1-2, and
- *     an L2 prefetch of the first routed weights once the selection is
- *     known); one persistent expert kernel that streams the shared expert's
- *     up projection first -- it needs nothing from the router, so it runs
- *     while the router is still working (programmatic dependent launch) --
- *     then the routed experts and the shared expert's down projection, and
- *     finishes with the combine (step 6): the CTA that completes a block of
- *     output columns writes it.  stream_aux is not used.  (With
- *     MOE_FLAG_TCGEN05 the combine is a third kernel.)
+ *   default: three kernels on stream_main.  The router kernel (steps 1-2);
+ *     one persistent expert kernel that streams the shared expert's up
+ *     projection first -- it needs nothing from the router, so it runs while
+ *     the router is still working (programmatic dependent launch) -- then the
+ *     routed experts and the shared expert's down projection; the combine
+ *     (step 6).  stream_aux is not used.
  *   MOE_FLAG_TWO_STREAM: the pages' layout.  Router and routed experts on
  *     stream_main, the shared expert on stream_aux (forked and joined with
  *     events), then a separate combine kernel.
@@ -85,8 +82,8 @@ extern "C" {
  * logits before softmax and selection; NULL means no bias.  It is read by
  * every forward (the pointer is kept, the data is not copied).
  * flags: any combination of MOE_FLAG_TWO_STREAM (see the top of this file),
- * MOE_FLAG_TCGEN05 and MOE_FLAG_TEST_HOLD_PANEL (below); other bits are
- * rejected with MOE_ERR_UNSUPPORTED_SHAPE.
+ * MOE_FLAG_TCGEN05, MOE_FLAG_TEST_HOLD_PANEL and MOE_FLAG_FP8_WEIGHTS
+ * (below); other bits are rejected with MOE_ERR_UNSUPPORTED_SHAPE.
  */
 #define MOE_FLAG_TWO_STREAM 1u
 /*
@@ -110,6 +107,17 @@ extern "C" {
  * path without faulting or hanging the GPU.
  */
 #define MOE_FLAG_TEST_HOLD_PANEL 4u
+/*
+ * MOE_FLAG_FP8_WEIGHTS: the expert weights (routed and shared) are 8-bit e4m3
+ * codes with fp32 block scales, passed to moe_decode_forward_fp8 (the other
+ * forward entry points reject such a handle).  Weight-only: the router and
+ * the activations stay bf16, products are taken in f16 x f16 -> fp32 (every
+ * e4m3 value and the activations are exact in f16) and each 128 x 128 block's
+ * partial sums are multiplied by its scale.  Needs hidden, inter and
+ * shared_inter to be multiples of 128; not combinable with MOE_FLAG_TCGEN05.
+ * An extension beyond the pages, which do not discuss weight precision.
+ */
+#define MOE_FLAG_FP8_WEIGHTS 8u
 typedef struct moe_decode_shapes {
   int32_t hidden;
   int32_t n_experts;
@@ -129,8 +137,8 @@ typedef struct moe_decode_ctx* moe_decode_t;
  *   forwards          : successful forwards enqueued by this handle
  *   kernels_launched  : kernels enqueued by this handle since creation
  *   last_kernels      : kernels enqueued by the last forward (default plan:
- *                       2, 3 with MOE_FLAG_TCGEN05; MOE_FLAG_TWO_STREAM:
- *                       4, or 3 without a shared expert)
+ *                       3; MOE_FLAG_TWO_STREAM: 4, or 3 without a shared
+ *                       expert)
  *   last_token_tiles  : token tiles of 8 the expert kernels were prepared for
  *                       in the last forward (ceil(min(batch, 32) / 8))
  * Device side (counted by the expert kernels as they run, cumulative since
@@ -205,13 +213,45 @@ int moe_decode_forward(moe_decode_t h, const void* x, const void* router_w,
  * registered memory on a unified-addressing system), the kernels store the
  * results into them directly; otherwise the results go through device
  * staging buffers and three device-to-host copies.  Pinned buffers give the
- * fastest transfers; pageable ones work.
+ * fastest transfers; pageable ones work.  When x_host is pinned too, the
+ * copy of x and the forward are captured once into a CUDA graph owned by
+ * the handle and replayed by later calls with the same arguments (every
+ * pointer, the batch, the streams and the wait limit); any change re-captures
+ * it.  (Not on the legacy default stream, not from a stream that is already
+ * being captured, and not while per-kernel timing events are set: those
+ * calls run eagerly.)
  */
 int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* router_w,
                             const void* const* w13, const void* const* w2,
                             const void* shared_w13, const void* shared_w2,
                             void* out_host, int32_t* ids_host, float* w_host,
                             int32_t batch, void* stream_main, void* stream_aux);
+
+/*
+ * moe_decode_forward with e4m3 expert weights (a handle created with
+ * MOE_FLAG_FP8_WEIGHTS).  x, router_w, out, topk_ids, topk_w, batch and the
+ * streams as for moe_decode_forward.  Each expert matrix is given in [out,
+ * in] layout -- every output's weights contiguous -- as uint8 e4m3 codes,
+ * with a float32 scale array [ceil(in / 128), P] row-major, P = 4 *
+ * ceil(ceil(out / 128) / 4) (rows padded to 16 bytes): the weight of
+ * (output o, input i) is decode(code[o, i]) * scale[i / 128, o / 128].
+ *   w13q  HOST array of n_experts device pointers -> uint8 [2*inter, hidden]
+ *         (outputs [0, inter) the gate, [inter, 2*inter) the up projection)
+ *   w13s  HOST array of n_experts device pointers -> float32 scales of w13q
+ *   w2q   HOST array of n_experts device pointers -> uint8 [hidden, inter]
+ *   w2s   HOST array of n_experts device pointers -> float32 scales of w2q
+ *   shared_w13q, shared_w13s, shared_w2q, shared_w2s: the shared expert's,
+ *         device pointers (NULL iff n_shared == 0)
+ * Code and scale arrays 16-byte aligned.  An all-ones exponent and mantissa
+ * (0x7F / 0xFF) is NaN in e4m3 and propagates.  Errors: as
+ * moe_decode_forward; MOE_ERR_INVALID_ARG also for a handle made without
+ * MOE_FLAG_FP8_WEIGHTS.
+ */
+int moe_decode_forward_fp8(moe_decode_t h, const void* x, const void* router_w, const void* const* w13q,
+                           const void* const* w13s, const void* const* w2q, const void* const* w2s,
+                           const void* shared_w13q, const void* shared_w13s, const void* shared_w2q,
+                           const void* shared_w2s, void* out, int32_t* topk_ids, float* topk_w, int32_t batch,
+                           void* stream_main, void* stream_aux);
 
 /* Free the workspace and events; NULL is accepted.  Waits for the handle's
  * work first, as moe_decode_get_status does. */
@@ -265,8 +305,7 @@ const char* moe_decode_last_cuda_error_string(void);
  *   [4] before the shared expert, [5] after it;
  * with the default plan (all on stream_main) [0] before the router, [1] and
  * [4] after it, [2] and [5] after the expert kernel (shared + routed
- * experts, and the combine, which it finishes with), [3] after the combine
- * (right after [2] unless MOE_FLAG_TCGEN05 runs it as its own kernel).  cudaEventElapsedTime gives each kernel's duration.  Recording an event
+ * experts), [3] after the combine.  cudaEventElapsedTime gives each kernel's duration.  Recording an event
  * between two kernels also makes the second wait for the first to finish
  * (no early launch), so timed forwards can be slightly slower.  The handle
  * keeps the array's values (not the pointer); the caller keeps the events

@@ -29,7 +29,9 @@ MOE_ERR_DEVICE_PLAN = -8
 
 # Entry points declared in include/moe_decode.h (checked by the tests).
 EXPORTED = (
-    "moe_decode_init", "moe_decode_forward", "moe_decode_forward_host", "moe_decode_destroy",
+    "moe_decode_init", "moe_decode_forward", "moe_decode_forward_host",
+    "moe_decode_forward_fp8",
+    "moe_decode_destroy",
     "moe_decode_get_status", "moe_decode_get_stats", "moe_decode_error_string",
     "moe_decode_last_cuda_error", "moe_decode_last_cuda_error_string", "moe_decode_workspace_bytes",
     "moe_decode_set_timing_events", "moe_decode_set_wait_limit", "moe_router_topk_noalloc",
@@ -39,6 +41,7 @@ MOE_TIMING_EVENTS = 6
 MOE_FLAG_TWO_STREAM = 1
 MOE_FLAG_TCGEN05 = 2
 MOE_FLAG_TEST_HOLD_PANEL = 4
+MOE_FLAG_FP8_WEIGHTS = 8
 
 
 class Shapes(ctypes.Structure):
@@ -88,6 +91,8 @@ def load_library() -> ctypes.CDLL:
     lib.moe_decode_forward.restype = I
     lib.moe_decode_forward_host.argtypes = fwd
     lib.moe_decode_forward_host.restype = I
+    lib.moe_decode_forward_fp8.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_int32, P, P]
+    lib.moe_decode_forward_fp8.restype = I
     lib.moe_decode_destroy.argtypes = [P]
     lib.moe_decode_destroy.restype = I
     lib.moe_decode_get_status.argtypes = [P]
@@ -163,20 +168,20 @@ def router_topk_noalloc_status(stream=None) -> int:
 class MoEDecode:
     """One MoE block shape bound to the current CUDA device (owns a workspace).
 
-    two_stream=False (default): router kernel and one expert kernel (shared
-    and routed experts, ending with the combine + residual) on the main
-    stream.  two_stream=True:
+    two_stream=False (default): router kernel, one expert kernel (shared
+    and routed experts) and the combine on the main stream.  two_stream=True:
     MOE_FLAG_TWO_STREAM, the shared expert on the aux stream.  tcgen05=True:
     MOE_FLAG_TCGEN05, the expert kernel on tcgen05 with TMEM accumulators."""
 
     def __init__(self, hidden: int, n_experts: int, top_k: int, inter: int, shared_inter: int = 0,
                  n_shared: int = 1, max_batch: int = 64, router_bias=None, two_stream: bool = False,
-                 tcgen05: bool = False, extra_flags: int = 0):
+                 tcgen05: bool = False, extra_flags: int = 0, fp8: bool = False):
         self._lib = load_library()
         self._bias = router_bias  # keep the device tensor alive
         self.two_stream = bool(two_stream)
         self.tcgen05 = bool(tcgen05)
         flags = (MOE_FLAG_TWO_STREAM if two_stream else 0) | (MOE_FLAG_TCGEN05 if tcgen05 else 0) | int(extra_flags)
+        flags |= MOE_FLAG_FP8_WEIGHTS if fp8 else 0
         self.shapes = Shapes(hidden, n_experts, top_k, inter, shared_inter if n_shared else 0, n_shared,
                              max_batch, _ptr(router_bias), flags)
         h = ctypes.c_void_p()
@@ -226,6 +231,22 @@ class MoEDecode:
                                           _ptr(shared_w13), _ptr(shared_w2), _ptr(out), _ptr(topk_ids),
                                           _ptr(topk_w), int(batch), sm, sa)
         _check(rc, "moe_decode_forward")
+
+    def forward_fp8(self, x, router_w, w13q, w13s, w2q, w2s, shared_w13q, shared_w13s, shared_w2q, shared_w2s,
+                    out, topk_ids, topk_w, batch: Optional[int] = None, stream_main=None, stream_aux=None):
+        """Enqueue one forward with e4m3 expert weights (handle made with
+        fp8=True): w13q/w2q [E, out, in] uint8 codes (or lists), w13s/w2s
+        their float32 block scales [E, ceil(in/128), padded ceil(out/128)]."""
+        import torch
+        if batch is None:
+            batch = x.shape[0]
+        sm = _stream_handle(stream_main if stream_main is not None else torch.cuda.current_stream())
+        sa = _stream_handle(stream_aux if stream_aux is not None else self.aux_stream())
+        rc = self._lib.moe_decode_forward_fp8(self._h, _ptr(x), _ptr(router_w), self._table(w13q), self._table(w13s),
+                                              self._table(w2q), self._table(w2s), _ptr(shared_w13q),
+                                              _ptr(shared_w13s), _ptr(shared_w2q), _ptr(shared_w2s), _ptr(out),
+                                              _ptr(topk_ids), _ptr(topk_w), int(batch), sm, sa)
+        _check(rc, "moe_decode_forward_fp8")
 
     def forward_host(self, x_host, router_w, w13, w2, shared_w13, shared_w2, out_host, ids_host, w_host,
                      batch: Optional[int] = None, stream_main=None, stream_aux=None):

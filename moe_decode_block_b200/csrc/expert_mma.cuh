@@ -97,6 +97,14 @@ __host__ __device__ constexpr int class_rows(int c) { return c == 0 ? 16 : (c ==
 __host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : 4); }
 // class of a unit with n <= kUnitTok tokens
 __host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : 2); }
+// FP8 (e4m3) weights: the same panel widths, stages of 32 rows (class 0,
+// 2048 x 32 = 64 KB) and 64 rows (classes 1 and 2: 64 KB and 32 KB), so the
+// accumulators per consumer warp are the same as for bf16 weights and the
+// tokens' activation rows fit the same buffer.
+__host__ __device__ constexpr int class_rows_fp8(int c) { return c == 0 ? 32 : 64; }
+__host__ __device__ constexpr int geo_rows(int c, bool fp8) { return fp8 ? class_rows_fp8(c) : class_rows(c); }
+// Bytes of the fp8 weights of a stage (the block scales follow them).
+constexpr int kFp8StageWBytes = 65536;
 // Consumer warps: sixteen in every instance (seventeen warps with the
 // producer cap a thread at 96 registers, room for the 32 accumulators).
 __host__ __device__ constexpr int consumer_warps_for(int) { return 16; }
@@ -171,9 +179,14 @@ struct MmaArgs {
   unsigned* panel_ready_s;
   unsigned* queue;           // [0] ticket counter, [1] finished CTAs (zero between calls), [2] launch epoch
   int* status;
-  unsigned long long* stage_counts;  // [kNumClasses * 2]: stages issued per (token class, UP / DOWN), cumulative
   uint32_t spin_limit;       // probes before a bounded wait gives up
   int hold_panel;            // testing only: routed UP panel whose publication is withheld (-1: none)
+  int stagger;               // segment B: stagger period of the first big chunks (0: none)
+  // FP8 weights: fp32 block scales, rows of sc_pitch* floats per 128 input
+  // rows (routed experts' scale arrays come in the pointer tables)
+  const float* sc13_s;       // shared expert w13 scales
+  const float* sc2_s;        // shared expert w2 scales
+  int sc_pitch13, sc_pitch13_s, sc_pitch2;
 };
 
 // Producer's copy of the plan in shared memory: per unit the expert id,
@@ -196,12 +209,12 @@ __host__ __device__ __forceinline__ int unit_panels(int cls, bool up, int H, int
   const int lw = class_lw(cls);
   return up ? (I + lw / 2 - 1) / (lw / 2) : (H + lw - 1) / lw;
 }
-__host__ __device__ __forceinline__ int unit_panel_stages(int cls, bool up, int H, int I) {
-  const int r = class_rows(cls);
+__host__ __device__ __forceinline__ int unit_panel_stages(int cls, bool up, int H, int I, bool fp8 = false) {
+  const int r = geo_rows(cls, fp8);
   return up ? (H + r - 1) / r : (I + r - 1) / r;
 }
-__host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int I) {
-  return unit_panels(cls, up, H, I) * unit_panel_stages(cls, up, H, I);
+__host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int I, bool fp8 = false) {
+  return unit_panels(cls, up, H, I) * unit_panel_stages(cls, up, H, I, fp8);
 }
 
 // Ticket schedule over a segment of T stages for a grid of G CTAs
@@ -211,9 +224,19 @@ __host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int
 // fraction of the list, because every chunk ends in a flush of the
 // consumers' partial sums.  make_round: one round of at most G chunks of
 // max(1, T / G) stages plus the remainder.
+// Staggered starts (stag = S > 1): the first G big chunks are shorter by
+// tk mod S stages, so CTAs that start the segment together reach their chunk
+// changes -- a flush and, for UP pieces, a fence -- at different times
+// instead of all at once; the stages taken off go to the quarter band.
 struct Sched {
-  int T, c_big, c_mid, n_big, n_mid, T1, T2, n_tickets;
+  int T, c_big, c_mid, n_big, n_mid, T1, T2, n_tickets, G, stag;
 };
+// stages taken off the first m big chunks (m <= G)
+__device__ __forceinline__ int sched_stagger_sum(int m, int S) {
+  if (S <= 1) return 0;
+  const int q = m / S, r = m - q * S;
+  return q * (S * (S - 1) / 2) + r * (r - 1) / 2;
+}
 __device__ __forceinline__ Sched make_round(int T, int G) {
   Sched s;
   s.T = T;
@@ -225,21 +248,25 @@ __device__ __forceinline__ Sched make_round(int T, int G) {
   s.n_mid = T - s.T1 > 0 ? 1 : 0;
   s.T2 = T;
   s.n_tickets = s.n_big + s.n_mid;
+  s.G = G;
+  s.stag = 0;
   return s;
 }
-__device__ __forceinline__ Sched make_sched(int T, int G, int div) {
+__device__ __forceinline__ Sched make_sched(int T, int G, int div, int stag = 0) {
   Sched s;
   s.T = T;
+  s.G = G;
   int c = T / (div * G);
   c = c < 1 ? 1 : (c > kMaxChunk ? kMaxChunk : c);
   s.c_big = c;
   s.c_mid = c / 4 < 1 ? 1 : c / 4;
+  s.stag = stag < c / 2 ? stag : c / 2;  // every big chunk keeps at least half its stages
   const int singles = T < 2 * G ? T : 2 * G;
   const int mid_max = 3 * G * s.c_mid;
   const int rest = T - singles;
   const int mid = rest < mid_max ? rest : mid_max;
   s.n_big = (rest - mid) / c;
-  s.T1 = s.n_big * c;
+  s.T1 = s.n_big * c - sched_stagger_sum(s.n_big < G ? s.n_big : G, s.stag);
   s.n_mid = (T - singles - s.T1) / s.c_mid;
   s.T2 = s.T1 + s.n_mid * s.c_mid;
   s.n_tickets = s.n_big + s.n_mid + (T - s.T2);
@@ -248,8 +275,8 @@ __device__ __forceinline__ Sched make_sched(int T, int G, int div) {
 // stages [b, e) of ticket tk (0 <= tk < n_tickets)
 __device__ __forceinline__ void sched_range(const Sched& s, int tk, int& b, int& e) {
   if (tk < s.n_big) {
-    b = tk * s.c_big;
-    e = b + s.c_big;
+    b = tk * s.c_big - sched_stagger_sum(tk < s.G ? tk : s.G, s.stag);
+    e = b + s.c_big - (tk < s.G && s.stag > 1 ? tk % s.stag : 0);
   } else if (tk - s.n_big < s.n_mid) {
     b = s.T1 + (tk - s.n_big) * s.c_mid;
     e = b + s.c_mid;
@@ -270,6 +297,40 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
 
 __device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Two e4m3 values (the low and high byte of the low 16 bits of v) to f16x2
+// (low byte -> low half); exact: every e4m3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_lo_to_f16x2(uint32_t v) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(d) : "r"(v));
+  return d;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2(uint32_t v) {
+  uint32_t d;
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, hi;\n\t}" : "=r"(d) : "r"(v));
+  return d;
+}
+// bf16x2 -> f16x2 (round to nearest; exact for the activations' range)
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(__uint_as_float(v & 0xffff0000u)), "f"(__uint_as_float(v << 16)));
+  return d;
+}
+
+__device__ __forceinline__ void mma_f16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -354,6 +415,100 @@ __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint
   }
 }
 
+// One stage of tensor-core work on e4m3 weights (class C geometry: LWc
+// columns x class_rows_fp8(C) rows), accumulated into the same fragments as
+// mma_stage.  The stage holds the weights as [32-row chunk][column][32 bytes
+// of rows] -- each column's rows contiguous, as the [out, in] layout stores
+// them -- with TMA's 32-byte swizzle (the 16-byte half of a 32-byte row is
+// XORed with bit 2 of the column index).  ldmatrix (b16, not transposed)
+// gives a lane (g, t) of an 8 x 8 tile the four bytes of rows 4t .. 4t+3 of
+// column g: converted to f16, its low pair is the A operand's first k pair
+// and its high pair the second, which is the k order (0 1 | 8 9 ...)
+// relabelled; the tokens' fragments are loaded in the same order (rows 4t ..
+// 4t+3 as b0, b1), so each product pairs the same row of both.  Every e4m3
+// value is exact in f16 and the activations (bf16, |v| well inside f16's
+// range) are converted to f16 too; the stage's partial products (fp32) are
+// multiplied by the warp's block scale -- all of a warp's columns and a
+// stage's rows lie in one 128 x 128 block -- and added to the accumulators.
+template <int C, int NF, int CW>
+__device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, uint32_t sx, const float* srow,
+                                              int LW, int nrows, int ntiles, bool up, int c0, int uoff, int I,
+                                              int warp, int lane) {
+  constexpr int LWc = class_lw(C), R = class_rows_fp8(C);
+  constexpr int MT = class_mt(C, CW), NT = class_nt(C), KC32 = R / 32;
+  static_assert(MT * NT <= NF, "accumulator budget");
+  constexpr int xpitch = R * 2 + 16;
+  const int m0 = warp * MT * 16;
+  if (m0 >= LW) return;
+  const int out0 = up ? (m0 < uoff ? c0 + m0 : I + c0 + (m0 - uoff)) : c0 + m0;
+  const float sc = srow[out0 >> 7];
+  const int g = lane >> 2, tq = lane & 3;
+  const int li = lane >> 3, lr = lane & 7;
+  // tokens' fragments of tile nt for this 32-row chunk: rows 4tq .. 4tq + 3
+  // of each 16-row half, converted to f16 (zero past the stage's rows)
+  auto load_b = [&](int kc, int nt, uint32_t (&b)[4]) {
+    const uint32_t a = sx + (uint32_t)(nt * 8 + g) * xpitch + (uint32_t)(kc * 32 + 4 * tq) * 2;
+    uint32_t v0, v1, v2, v3;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(a));
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v2), "=r"(v3) : "r"(a + 32));
+    const bool h0 = kc * 32 + 4 * tq < nrows, h1 = kc * 32 + 16 + 4 * tq < nrows;
+    b[0] = h0 ? bf16x2_to_f16x2(v0) : 0u;
+    b[1] = h0 ? bf16x2_to_f16x2(v1) : 0u;
+    b[2] = h1 ? bf16x2_to_f16x2(v2) : 0u;
+    b[3] = h1 ? bf16x2_to_f16x2(v3) : 0u;
+  };
+  // one token tile: its fragments stay in registers for all m-tiles; more
+  // tiles: reloaded per m-tile (keeping them all costs spills)
+  constexpr bool kKeepB = NT == 1;
+  // (the chunk loop stays rolled: unrolled, its hoisted addresses and
+  // fragments spill in the classes with several token tiles)
+#pragma unroll 1
+  for (int kc = 0; kc < KC32; ++kc) {
+    if (kc * 32 >= nrows) break;
+    uint32_t bk[4] = {0u, 0u, 0u, 0u};
+    if (kKeepB) load_b(kc, 0, bk);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      if (m0 + mt * 16 < LW) {
+        const int col = m0 + mt * 16 + (li & 1) * 8 + lr;   // local column of this lane's ldmatrix row
+        const int half = (li >> 1) ^ ((col >> 2) & 1);       // 32-byte swizzle
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(sw + (uint32_t)(kc * LWc * 32 + col * 32 + half * 16), r0, r1, r2, r3);
+        if (kKeepB) {
+          float t[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_f16_16816(t, e4m3x2_lo_to_f16x2(r0), e4m3x2_lo_to_f16x2(r1), e4m3x2_hi_to_f16x2(r0),
+                        e4m3x2_hi_to_f16x2(r1), bk[0], bk[1]);
+          mma_f16_16816(t, e4m3x2_lo_to_f16x2(r2), e4m3x2_lo_to_f16x2(r3), e4m3x2_hi_to_f16x2(r2),
+                        e4m3x2_hi_to_f16x2(r3), bk[2], bk[3]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[mt * NT][j] = fmaf(sc, t[j], acc[mt * NT][j]);
+        } else {
+          // half by half: one half's A fragment and one tile's B pair live
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t ra = hf ? r2 : r0, rb = hf ? r3 : r1;
+            const uint32_t a0 = e4m3x2_lo_to_f16x2(ra), a1 = e4m3x2_lo_to_f16x2(rb);
+            const uint32_t a2 = e4m3x2_hi_to_f16x2(ra), a3 = e4m3x2_hi_to_f16x2(rb);
+            const bool live = kc * 32 + hf * 16 + 4 * tq < nrows;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              if (nt < ntiles) {
+                const uint32_t ad = sx + (uint32_t)(nt * 8 + g) * xpitch + (uint32_t)(kc * 32 + hf * 16 + 4 * tq) * 2;
+                uint32_t v0, v1;
+                asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(ad));
+                float t[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_f16_16816(t, a0, a1, a2, a3, live ? bf16x2_to_f16x2(v0) : 0u, live ? bf16x2_to_f16x2(v1) : 0u);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[mt * NT + nt][j] = fmaf(sc, t[j], acc[mt * NT + nt][j]);
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 // Local columns of a stage: DOWN [0, w) -> c0 + l; UP gate [0, w) -> c0 + l
 // and up [uoff, uoff + w) -> I + c0 + (l - uoff); anything else is padding.
 // w and uoff are multiples of 8, so four consecutive local columns map to four
@@ -416,8 +571,7 @@ struct SmemView {
   uint64_t* empty;
   StageHdr* hdr;
   volatile int* s_misc;  // [0]: abort flag (a bounded wait gave up), [1]: wait limit (probes),
-                         // [2]: stages issued,
-                         // [4 + 2 * cls + (DOWN ? 1 : 0)]: stages issued per token class
+                         // [2]: stages issued
   uint16_t* s_uexp;      // [kMaxUnits]
   uint16_t* s_ubeg;      // [kMaxUnits]
   uint16_t* s_aslot;     // [kMaxAssign]
@@ -445,7 +599,7 @@ __device__ __forceinline__ SmemView carve_smem(uint8_t* raw, int NS) {
 // The producer warp: takes tickets, walks the work list and fills the stage
 // ring (weights by TMA, the stage's token activations, the stage header);
 // ends by posting a kKindEnd header.  Shared by both expert kernels.
-template <int KC, bool TMAP>
+template <int KC, bool TMAP, bool FP8 = false>
 __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertTable& tab13, const ExpertTable& tab2,
                                               const SmemView& sv, int NS, unsigned ready_mark, int lane) {
   uint8_t* stages = sv.stages;
@@ -480,13 +634,13 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
     int S_up = 0, S_dn = 0;
     for (int su = 0; su < args.n_su; ++su) {
       const int c = cls_of(su_tokens(su));
-      S_up += unit_stages(c, true, H, args.Is);
-      S_dn += unit_stages(c, false, H, args.Is);
+      S_up += unit_stages(c, true, H, args.Is, FP8);
+      S_dn += unit_stages(c, false, H, args.Is, FP8);
     }
     const int S_A = S_up;  // segment A: the shared UP stages
     const Sched sch_A = make_round(S_up, G);
     // segment B: the routed units, read from the plan once a ticket reaches it
-    Sched sch_B = make_sched(S_dn, G, 4);
+    Sched sch_B = make_sched(S_dn, G, 4, args.stagger);
     bool b_known = !args.has_routed;
     int n_units_r = 0;
     auto know_b = [&]() {
@@ -518,7 +672,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         s_uexp[u] = (uint16_t)ex;
         s_ubeg[u] = (uint16_t)bg;
         const int c = cls_of(cnt);
-        T += unit_stages(c, true, H, args.I) + unit_stages(c, false, H, args.I);
+        T += unit_stages(c, true, H, args.I, FP8) + unit_stages(c, false, H, args.I, FP8);
       }
       for (int i = lane; i < nas; i += 32) {
         int sl = __ldcg(&pl->assign_slot[i]);
@@ -532,7 +686,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) T += __shfl_xor_sync(0xffffffffu, T, off);
       __syncwarp();
-      sch_B = make_sched(T + S_dn, G, 4);
+      sch_B = make_sched(T + S_dn, G, 4, args.stagger);
       b_known = true;
     };
     // Cursor over the work list: group (0 shared UP, 1 routed UP, 2 shared
@@ -544,8 +698,8 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
     int cur_g = 0, cur_unit = 0, cur_base = 0, cur_size = 0;
     auto group_units = [&](int g) { return g_seg(g) == 0 ? args.n_su : n_units_r; };
     auto unit_size = [&](int g, int u) {
-      return g_seg(g) == 0 ? unit_stages(cls_of(su_tokens(u)), g_up(g), H, args.Is)
-                           : unit_stages(cls_of(plan_tokens(u)), g_up(g), H, args.I);
+      return g_seg(g) == 0 ? unit_stages(cls_of(su_tokens(u)), g_up(g), H, args.Is, FP8)
+                           : unit_stages(cls_of(plan_tokens(u)), g_up(g), H, args.I, FP8);
     };
     if (args.n_su > 0) cur_size = unit_size(0, 0);
     auto advance = [&]() {
@@ -624,8 +778,8 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
           }
           u_cls = cls_of(u_ntok);
           u_lw = class_lw(u_cls);
-          u_R = class_rows(u_cls);
-          u_S = unit_panel_stages(u_cls, up, H, u_I);
+          u_R = geo_rows(u_cls, FP8);
+          u_S = unit_panel_stages(u_cls, up, H, u_I, FP8);
         }
         const int ntok = u_ntok, cls = u_cls, lw = u_lw, R = u_R, S = u_S, Iu = u_I;
         const int loc = t - cur_base;
@@ -685,8 +839,13 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         // tensor-map path: loads = halves x 16-row blocks x groups of 4 chunks
         const int t_ncg = (w / kChunkCols + kBoxChunks - 1) / kBoxChunks;
         const int t_nrb = R / kBoxRows;
-        const int t_nops = (up ? 2 : 1) * t_nrb * t_ncg;
-        const uint32_t wtotal = TMAP ? (uint32_t)t_nops * kBoxBytes : (uint32_t)nrows * (up ? 2u : 1u) * wbytes;
+        // FP8: loads = halves x 256-column blocks x 32-row chunks, plus the
+        // stage's row of block scales (pitch floats per 128 weight rows)
+        const int f_nmb = (w + 255) / 256, f_per_half = f_nmb * (R / 32);
+        const int f_pitch = up ? (seg == 0 ? args.sc_pitch13_s : args.sc_pitch13) : args.sc_pitch2;
+        const int t_nops = FP8 ? (up ? 2 : 1) * f_per_half : (up ? 2 : 1) * t_nrb * t_ncg;
+        const uint32_t wtotal = FP8 ? (uint32_t)t_nops * kBoxBytes + (uint32_t)f_pitch * 4u
+                                    : (TMAP ? (uint32_t)t_nops * kBoxBytes : (uint32_t)nrows * (up ? 2u : 1u) * wbytes);
         const uint32_t bytes = wtotal + (uint32_t)ntok * nrows * 2;
         uint8_t* sw = stages + (size_t)slot * kStageBytesMma;
         uint8_t* sx = sw + kStageWBytes;
@@ -713,7 +872,20 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         // activations of this lane's token: x row (UP) or a row (DOWN)
         const void* act = up ? (const void*)(args.x + (size_t)u_src * H + row0)
                              : (const void*)((seg == 0 ? args.a_s : args.a) + (size_t)u_src * Iu + row0);
-        if (TMAP) {
+        if constexpr (FP8) {
+          // [32-row chunk][column][32 bytes] with 32-byte swizzle, UP's up
+          // half from local column lw / 2 (the weights are [out, in])
+          for (int o = lane; o < t_nops; o += 32) {
+            const int hh = o / f_per_half, rem = o - hh * f_per_half;
+            const int kc = rem / f_nmb, mb = rem - kc * f_nmb;
+            uint8_t* dst = sw + (size_t)kc * lw * 32 + (size_t)(hh * (lw / 2) + mb * 256) * 32;
+            const int m = (up ? (hh ? Iu + c0 : c0) : c0) + mb * 256;
+            tma_load_2d(dst, u_map, row0 + kc * 32, m, &full[slot], pol);
+          }
+          if (lane == 31)  // u_W holds the matrix's scale array here
+            bulk_copy_g2s(sw + kFp8StageWBytes, reinterpret_cast<const float*>(u_W) + (size_t)(row0 >> 7) * f_pitch,
+                          (uint32_t)f_pitch * 4u, &full[slot], pol);
+        } else if (TMAP) {
           const int per_half = t_nrb * t_ncg;
           const int rbstride = (lw / kChunkCols) * kChunkTile;
           const int nch_half = (up ? lw / 2 : lw) / kChunkCols;
@@ -738,7 +910,6 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         if (lane < ntok) bulk_copy_g2s_plain(sx + (size_t)lane * xpitch, act, (uint32_t)nrows * 2, &full[slot]);
         if (lane == 0) {
           s_misc[2] = (int)(q + 1);
-          s_misc[4 + 2 * cls + (up ? 0 : 1)] += 1;
         }
       }
       if (stop) break;
@@ -759,7 +930,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
     __syncwarp();
 }
 
-template <int KC, bool TMAP>
+template <int KC, bool TMAP, bool FP8 = false>
 __global__ void __launch_bounds__(expert_threads(KC), 1)
     expert_mlp_kernel(const __grid_constant__ MmaArgs args, const __grid_constant__ ExpertTable tab13,
                       const __grid_constant__ ExpertTable tab2) {
@@ -795,7 +966,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   const unsigned ready_mark = __ldcg(&args.queue[2]) + 1u;
 
   if (is_producer) {
-    producer_loop<KC, TMAP>(args, tab13, tab2, sv, NS, ready_mark, lane);
+    producer_loop<KC, TMAP, FP8>(args, tab13, tab2, sv, NS, ready_mark, lane);
   } else {
     // =============================================================== consumers
     // (they read nothing the router writes: the stage headers carry it)
@@ -809,9 +980,11 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       const bool landed = mbar_wait_abortable_warp(&full[slot], ph, args.status, abort_flag);
       if (!landed) break;
       // the header stays valid until this warp releases the slot (below,
-      // once the stage's tensor-core work is done)
+      // once the stage's tensor-core work is done); every lane reads the same
+      // word, written before the phase the warp observed, so the branch is
+      // uniform
       const StageHdr& hd = hdr[slot];
-      if (__shfl_sync(0xffffffffu, hd.kind, 0) == kKindEnd) break;
+      if (hd.kind == kKindEnd) break;
       const bool up = hd.kind == kKindUp;
       const bool sh = hd.seg == 0;
       const int Iu = sh ? args.Is : args.I;
@@ -830,13 +1003,25 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       }
       const uint32_t sw = smem_addr(stages + (size_t)slot * kStageBytesMma);
       const uint32_t sx = sw + kStageWBytes;
-      if (hd.cls == 0)
-        mma_stage<0, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-      else if constexpr (KC >= 1) {
-        if (hd.cls == 1)
-          mma_stage<1, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
-        else if constexpr (KC >= 2)
-          mma_stage<2, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+      if constexpr (FP8) {
+        const float* srow = reinterpret_cast<const float*>(stages + (size_t)slot * kStageBytesMma + kFp8StageWBytes);
+        if (hd.cls == 0)
+          mma_stage_fp8<0, NF, CW>(acc, sw, sx, srow, LW, hd.nrows, ntiles, up, c0, uoff, Iu, warp, lane);
+        else if constexpr (KC >= 1) {
+          if (hd.cls == 1)
+            mma_stage_fp8<1, NF, CW>(acc, sw, sx, srow, LW, hd.nrows, ntiles, up, c0, uoff, Iu, warp, lane);
+          else if constexpr (KC >= 2)
+            mma_stage_fp8<2, NF, CW>(acc, sw, sx, srow, LW, hd.nrows, ntiles, up, c0, uoff, Iu, warp, lane);
+        }
+      } else {
+        if (hd.cls == 0)
+          mma_stage<0, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+        else if constexpr (KC >= 1) {
+          if (hd.cls == 1)
+            mma_stage<1, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+          else if constexpr (KC >= 2)
+            mma_stage<2, NF, TMAP, CW>(acc, sw, sx, LW, hd.nrows, ntiles, warp, lane);
+        }
       }
       const bool piece_end = (hd.flags & kLast) != 0;
       // What the flush and the SwiGLU fix-up need from the header goes to
@@ -873,7 +1058,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
           unsigned* pcnt = sh ? args.panel_cnt_s : args.panel_cnt;
           unsigned* pready = sh ? args.panel_ready_s : args.panel_ready;
           const int panel = unit * (sh ? args.panel_stride_s : args.panel_stride) + cp;
-          const unsigned target = (unsigned)unit_panel_stages(cls, true, H, Iu) * CW;
+          const unsigned target = (unsigned)unit_panel_stages(cls, true, H, Iu, FP8) * CW;
           int last = 0;
           if (lane == 0 && !*abort_flag) {
             const unsigned steps = (unsigned)pstages;
@@ -929,8 +1114,6 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       mbar_wait_bounded(&full[qq % NS], (uint32_t)(qq / NS) & 1u, args.status);
   }
   if (tid == 0) {
-    for (int i = 0; i < 2 * kNumClasses; ++i)
-      if (s_misc[4 + i]) atomicAdd(&args.stage_counts[i], (unsigned long long)s_misc[4 + i]);
     // the last CTA out returns the counters to zero and advances the epoch
     __threadfence();
     const unsigned done = atomicAdd(&args.queue[1], 1u);

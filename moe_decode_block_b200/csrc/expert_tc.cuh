@@ -420,8 +420,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_wait_bounded(&full[qq % NS], (uint32_t)(qq / NS) & 1u, args.status);
   }
   if (tid == 0) {
-    for (int i = 0; i < 2 * kNumClasses; ++i)
-      if (s_misc[4 + i]) atomicAdd(&args.stage_counts[i], (unsigned long long)s_misc[4 + i]);
     __threadfence();
     const unsigned done = atomicAdd(&args.queue[1], 1u);
     if (done == gridDim.x - 1) {

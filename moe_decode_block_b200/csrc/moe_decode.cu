@@ -4,14 +4,11 @@
 // "Recovering time between operators": the shared expert overlaps routing,
 // weights are fetched before their consumer starts, the residual add is
 // fused into the producing epilogue, fewer launches per layer):
-//   default (two kernels, stream_main only):
-//     router+top-k+plan (+ L2 prefetch of the first routed stages); the
-//     persistent expert kernel, which streams the shared expert's up
-//     projection before its grid-dependency wait (so it overlaps the router),
-//     then the routed experts and the shared expert's down projection, and
-//     ends with the combine + residual (the CTA that completes an output
-//     column block writes it).  With MOE_FLAG_TCGEN05 the combine is a third
-//     kernel.
+//   default (three kernels, stream_main only):
+//     router+top-k+plan; the persistent expert kernel, which streams the
+//     shared expert's up projection before its grid-dependency wait (so it
+//     overlaps the router) and then the routed experts and the shared
+//     expert's down projection; combine + residual.
 //   MOE_FLAG_TWO_STREAM (four kernels, the pages' layout):
 //     stream_main: router, routed experts, [join] combine
 //     stream_aux : shared expert, forked with an event after the router
@@ -53,10 +50,19 @@ thread_local int g_last_cuda_error = 0;
 // state never destroys them.
 struct WorkspaceLayout {
   size_t status, ticket, router_epoch, logits, plan, h, a, panel_cnt, panel_ready, queue, h_s, a_s, panel_cnt_s, panel_ready_s,
-      queue_s, acc, cb_cnt, x_stage, out_stage, ids_stage, w_stage, state_end, maps, stage_counts, total;
+      queue_s, acc, x_stage, out_stage, ids_stage, w_stage, state_end, maps, stage_counts, total;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Block scales of e4m3 expert weights (moe_decode_forward_fp8).
+struct Fp8Scales {
+  const void* const* w13s;  // host array of E device pointers
+  const void* const* w2s;
+  const void* sw13s;        // shared expert
+  const void* sw2s;
+};
+
 inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 bool shapes_valid(const moe_decode_shapes* s) {
@@ -69,7 +75,13 @@ bool shapes_valid(const moe_decode_shapes* s) {
   if (s->n_shared != 0 && s->n_shared != 1) return false;
   if (s->n_shared == 1 && (!in(s->shared_inter, 8, 16384) || s->shared_inter % 8)) return false;
   if (!in(s->max_batch, 1, moe::kMaxBatch)) return false;
-  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05 | MOE_FLAG_TEST_HOLD_PANEL)) != 0) return false;
+  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05 | MOE_FLAG_TEST_HOLD_PANEL | MOE_FLAG_FP8_WEIGHTS)) != 0)
+    return false;
+  if (s->flags & MOE_FLAG_FP8_WEIGHTS) {
+    // e4m3 weights: whole 128 x 128 scale blocks, on the mma.sync kernel
+    if (s->hidden % 128 || s->inter % 128 || (s->n_shared && s->shared_inter % 128)) return false;
+    if (s->flags & MOE_FLAG_TCGEN05) return false;
+  }
   return true;
 }
 
@@ -116,7 +128,6 @@ WorkspaceLayout layout_for(const moe_decode_shapes* s) {
   L.panel_ready_s = take(su * ncp_s * 4 + 4);
   L.queue_s = take(4 * 4);
   L.acc = take(B * H * 4);
-  L.cb_cnt = take(moe::kMaxColBlocks * sizeof(unsigned));
   L.x_stage = take(B * H * 2);
   L.out_stage = take(B * H * 2);
   L.ids_stage = take(B * k * 4);
@@ -169,6 +180,14 @@ MlpKernel pick_mlp_t(int kc) {
   }
 }
 MlpKernel pick_mlp(int kc, bool tmap) { return tmap ? pick_mlp_t<true>(kc) : pick_mlp_t<false>(kc); }
+// The expert kernel on e4m3 weights (tensor-map path only).
+MlpKernel pick_mlp_fp8(int kc) {
+  switch (kc) {
+    case 0: return moe::expert_mlp_kernel<0, true, true>;
+    case 1: return moe::expert_mlp_kernel<1, true, true>;
+    default: return moe::expert_mlp_kernel<2, true, true>;
+  }
+}
 
 // Token class the expert kernel is compiled for at this batch: units hold
 // at most kMaxUnitTokens tokens.
@@ -212,6 +231,30 @@ bool encode_matrix_map(uint8_t* out, const void* base, int rows, int cols) {
   return true;
 }
 
+// Tensor map of an e4m3 matrix [rows, cols] stored row-major ([out, in]: a
+// row holds one output's weights over the inputs), seen as the 2-D tensor
+// {cols, rows} with {32, 256} boxes (32 bytes of inputs x 256 outputs) and
+// 32-byte swizzling (see mma_stage_fp8).
+bool encode_fp8_map(uint8_t* out, const void* base, int rows, int cols) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc || cols % 16) return false;
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols};
+  cuuint32_t box[2] = {32, 256};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return false;
+  std::memcpy(out, &m, sizeof m);
+  return true;
+}
+
+// Floats per row of an e4m3 matrix's block scales: one per 128 outputs,
+// padded to a multiple of 4 (16-byte rows).
+inline int scale_pitch(int outs) { return ((outs + 127) / 128 + 3) / 4 * 4; }
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
@@ -240,8 +283,7 @@ struct moe_decode_ctx {
   int grid_routed = 0, grid_shared = 0, grid_router_max = 0;
   bool grid_routed_auto = true;
   int router_chunk_rows = 0;
-  int prefetch_stages = 0;  // L2 prefetch by the router: stages of each first expert-kernel chunk
-  int lookahead = 0;        // expert kernel: L2 prefetch of the stage this many positions ahead
+  int stagger = 8;             // expert kernel: stagger period of the first segment-B chunks
   WorkspaceLayout L{};
   uint8_t* ws = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
@@ -286,7 +328,7 @@ int router_grid(const moe_decode_ctx* h, int /*batch*/) {
 }
 
 // Router kernel holding E <= 32 * NV logits per lane during top-k.
-using RouterKernel = void (*)(RouterArgs, ExpertTable);
+using RouterKernel = void (*)(RouterArgs);
 RouterKernel pick_router(int n_experts) {
   if (n_experts <= 128) return moe::router_topk_kernel<4>;
   if (n_experts <= 256) return moe::router_topk_kernel<8>;
@@ -319,21 +361,32 @@ int shared_grid(const moe_decode_ctx* h, int batch) {
   return g;
 }
 
+// A kernel's dynamic shared-memory limit is a property of the function, not
+// of a handle: raise it to what this handle needs, never lower it (another
+// handle, made for a larger batch, may rely on the higher limit).
+template <typename K>
+cudaError_t raise_smem_limit(K kern, int bytes) {
+  cudaFuncAttributes fa{};
+  cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.maxDynamicSharedSizeBytes >= bytes) return cudaSuccess;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
 int set_kernel_attrs(const moe_decode_ctx* h) {
   const int smem = (int)moe::mma_smem_bytes(h->n_stages);
   cudaError_t e;
   for (int kc = 0; kc < moe::kNumClasses; ++kc) {
     for (int tm = 0; tm < 2; ++tm) {
-      e = cudaFuncSetAttribute(pick_mlp(kc, tm), cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return fail_cuda(e);
+      if ((e = raise_smem_limit(pick_mlp(kc, tm), smem)) != cudaSuccess) return fail_cuda(e);
     }
   }
-  e = cudaFuncSetAttribute(moe::expert_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)moe::tc_smem_bytes(h->n_stages_tc));
-  if (e != cudaSuccess) return fail_cuda(e);
+  for (int kc = 0; kc < moe::kNumClasses; ++kc)
+    if ((e = raise_smem_limit(pick_mlp_fp8(kc), smem)) != cudaSuccess) return fail_cuda(e);
+  if ((e = raise_smem_limit(moe::expert_tc_kernel, (int)moe::tc_smem_bytes(h->n_stages_tc))) != cudaSuccess)
+    return fail_cuda(e);
   const int rsmem = (int)moe::router_smem_bytes(h->s.max_batch, h->s.n_experts, h->router_chunk_rows);
-  e = cudaFuncSetAttribute(pick_router(h->s.n_experts), cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem);
-  if (e != cudaSuccess) return fail_cuda(e);
+  if ((e = raise_smem_limit(pick_router(h->s.n_experts), rsmem)) != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }
 
@@ -344,30 +397,38 @@ int refresh_maps(moe_decode_ctx* h, const void* const* w13, const void* const* w
                  const void* sw2, cudaStream_t sm) {
   const moe_decode_shapes& s = h->s;
   const int E = s.n_experts;
+  const size_t nm = 2 * (size_t)E + 2, mb = moe::kTensorMapBytes;
+  const void** ptrs = h->map_ptrs.data();
+  uint8_t* stage = h->maps_host;
   bool changed = !h->maps_uploaded;
-  for (int e = 0; e < E && !changed; ++e) changed = (h->map_ptrs[e] != w13[e] || h->map_ptrs[E + e] != w2[e]);
-  if (s.n_shared && !changed) changed = (h->map_ptrs[2 * E] != sw13 || h->map_ptrs[2 * E + 1] != sw2);
+  for (int e = 0; e < E && !changed; ++e) changed = (ptrs[e] != w13[e] || ptrs[E + e] != w2[e]);
+  if (s.n_shared && !changed) changed = (ptrs[2 * E] != sw13 || ptrs[2 * E + 1] != sw2);
   if (!changed) return MOE_OK;
   cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
   cudaStreamIsCapturing(sm, &cap);
   // the staging buffer may still feed the previous upload
   if (h->maps_uploaded && cap == cudaStreamCaptureStatusNone) cudaEventSynchronize(h->ev_maps);
-  const size_t mb = moe::kTensorMapBytes;
+  const bool fp8 = (s.flags & MOE_FLAG_FP8_WEIGHTS) != 0;
+  // bf16: w13 [H, 2I], w2 [I, H]; e4m3: w13 [2I, H], w2 [H, I]
+  auto enc = [&](uint8_t* o, const void* p, int rows_bf16, int cols_bf16) {
+    return fp8 ? encode_fp8_map(o, p, cols_bf16, rows_bf16) : encode_matrix_map(o, p, rows_bf16, cols_bf16);
+  };
   for (int e = 0; e < E; ++e) {
-    if (!encode_matrix_map(h->maps_host + e * mb, w13[e], s.hidden, 2 * s.inter)) return MOE_ERR_INVALID_ARG;
-    if (!encode_matrix_map(h->maps_host + (E + e) * mb, w2[e], s.inter, s.hidden)) return MOE_ERR_INVALID_ARG;
-    h->map_ptrs[e] = w13[e];
-    h->map_ptrs[E + e] = w2[e];
+    if (!enc(stage + e * mb, w13[e], s.hidden, 2 * s.inter)) return MOE_ERR_INVALID_ARG;
+    if (!enc(stage + (E + e) * mb, w2[e], s.inter, s.hidden)) return MOE_ERR_INVALID_ARG;
+    ptrs[e] = w13[e];
+    ptrs[E + e] = w2[e];
   }
   if (s.n_shared) {
-    if (!encode_matrix_map(h->maps_host + 2 * E * mb, sw13, s.hidden, 2 * s.shared_inter)) return MOE_ERR_INVALID_ARG;
-    if (!encode_matrix_map(h->maps_host + (2 * E + 1) * mb, sw2, s.shared_inter, s.hidden)) return MOE_ERR_INVALID_ARG;
-    h->map_ptrs[2 * E] = sw13;
-    h->map_ptrs[2 * E + 1] = sw2;
+    if (!enc(stage + 2 * E * mb, sw13, s.hidden, 2 * s.shared_inter)) return MOE_ERR_INVALID_ARG;
+    if (!enc(stage + (2 * E + 1) * mb, sw2, s.shared_inter, s.hidden)) return MOE_ERR_INVALID_ARG;
+    ptrs[2 * E] = sw13;
+    ptrs[2 * E + 1] = sw2;
   }
-  cudaError_t e = cudaMemcpyAsync(h->ws + h->L.maps, h->maps_host, (2 * E + 2) * mb, cudaMemcpyHostToDevice, sm);
+  cudaError_t e = cudaMemcpyAsync(h->ws + h->L.maps, stage, nm * mb, cudaMemcpyHostToDevice, sm);
   if (e != cudaSuccess) return fail_cuda(e);
-  if (cap == cudaStreamCaptureStatusNone && (e = cudaEventRecord(h->ev_maps, sm)) != cudaSuccess) return fail_cuda(e);
+  if (cap == cudaStreamCaptureStatusNone && (e = cudaEventRecord(h->ev_maps, sm)) != cudaSuccess)
+    return fail_cuda(e);
   h->maps_uploaded = true;
   return MOE_OK;
 }
@@ -375,7 +436,8 @@ int refresh_maps(moe_decode_ctx* h, const void* const* w13, const void* const* w
 // Enqueue the whole forward (device pointers only).
 int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, const void* const* w13,
                     const void* const* w2, const void* shared_w13, const void* shared_w2, void* out,
-                    int32_t* topk_ids, float* topk_w, int batch, cudaStream_t sm, cudaStream_t sa) {
+                    int32_t* topk_ids, float* topk_w, int batch, cudaStream_t sm, cudaStream_t sa,
+                    const Fp8Scales* f8) {
   const moe_decode_shapes& s = h->s;
   cudaError_t e;
   int kernels = 0;
@@ -386,9 +448,11 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     if (e != cudaSuccess) return fail_cuda(e);
     h->dirty = false;
   }
+  // pointer tables (kernel parameters): the weights, or with e4m3 weights
+  // (read through their tensor maps) the block-scale arrays
   for (int i = 0; i < s.n_experts; ++i) {
-    h->tab13->p[i] = static_cast<const __nv_bfloat16*>(w13[i]);
-    h->tab2->p[i] = static_cast<const __nv_bfloat16*>(w2[i]);
+    h->tab13->p[i] = static_cast<const __nv_bfloat16*>(f8 ? f8->w13s[i] : w13[i]);
+    h->tab2->p[i] = static_cast<const __nv_bfloat16*>(f8 ? f8->w2s[i] : w2[i]);
   }
   if (h->use_tmap) {
     const int rc = refresh_maps(h, w13, w2, shared_w13, shared_w2, sm);
@@ -401,10 +465,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   const bool fork = two_stream && s.n_shared && sa != sm;
   const int n_su = shared_units(s, batch);
   const int kc = kernel_class(batch);
-  const MlpKernel mlp = h->use_tc ? moe::expert_tc_kernel : pick_mlp(kc, h->use_tmap);
-  // default plan on mma.sync: the combine + residual runs inside the expert
-  // kernel (the CTA that completes an output column block writes it)
-  const bool fused_combine = !two_stream && !h->use_tc;
+  const MlpKernel mlp = f8 ? pick_mlp_fp8(kc) : (h->use_tc ? moe::expert_tc_kernel : pick_mlp(kc, h->use_tmap));
   const int mlp_threads = h->use_tc ? moe::kTcThreads : moe::expert_threads(kc);
   const int n_stages = h->use_tc ? h->n_stages_tc : h->n_stages;
   const size_t smem = h->use_tc ? moe::tc_smem_bytes(n_stages) : moe::mma_smem_bytes(n_stages);
@@ -429,8 +490,11 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.max_units = (int)max_units(&s);
   base.panel_stride = moe::max_up_panels(s.inter);
   base.panel_stride_s = s.n_shared ? moe::max_up_panels(s.shared_inter) : 0;
-  base.w13_s = static_cast<const __nv_bfloat16*>(shared_w13);
-  base.w2_s = static_cast<const __nv_bfloat16*>(shared_w2);
+  base.w13_s = static_cast<const __nv_bfloat16*>(f8 ? f8->sw13s : shared_w13);
+  base.w2_s = static_cast<const __nv_bfloat16*>(f8 ? f8->sw2s : shared_w2);
+  base.sc_pitch13 = scale_pitch(2 * s.inter);
+  base.sc_pitch13_s = s.n_shared ? scale_pitch(2 * s.shared_inter) : 4;
+  base.sc_pitch2 = scale_pitch(s.hidden);
   base.maps13 = maps;
   base.maps2 = maps + (size_t)s.n_experts * mb;
   base.maps13_s = maps + 2 * (size_t)s.n_experts * mb;
@@ -448,9 +512,8 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.panel_ready_s = h->at<unsigned>(h->L.panel_ready_s);
   base.queue = h->at<unsigned>(h->L.queue);
   base.status = status;
-  base.stage_counts = h->at<unsigned long long>(h->L.stage_counts);
-  base.lookahead = h->use_tmap ? h->lookahead : 0;
   base.spin_limit = h->spin_limit;
+  base.stagger = h->stagger;
   // testing only: the handle's first forward withholds routed UP panel 0
   base.hold_panel = ((s.flags & MOE_FLAG_TEST_HOLD_PANEL) && h->stats.forwards == 0) ? 0 : -1;
 
@@ -474,65 +537,51 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   ra.topk_w = topk_w;
   ra.status = status;
   ra.spin_limit = h->spin_limit;
-  // the expert kernel that streams the routed units, for the router's L2
-  // prefetch of its first stages
-  {
-    const bool tw = (s.flags & MOE_FLAG_TWO_STREAM) != 0;
-    int g_exp = h->grid_routed;
-    if (tw && s.n_shared && sa != sm && h->grid_routed_auto) g_exp = h->num_sms - shared_grid(h, batch);
-    ra.prefetch_stages = h->prefetch_stages;
-    ra.expert_grid = g_exp < 1 ? 1 : g_exp;
-    ra.expert_kc = h->use_tc ? moe::kNumClasses - 1 : kc;
-    ra.inter = s.inter;
-    int sdn = 0;
-    if (!tw) {
-      for (int su = 0; su < n_su; ++su) {
-        const int n = std::min(moe::kMaxUnitTokens, batch - su * moe::kMaxUnitTokens);
-        const int c = std::min(moe::class_for_tokens(n), ra.expert_kc);
-        sdn += moe::unit_stages(c, false, s.hidden, s.shared_inter);
-      }
-    }
-    ra.shared_down_stages = sdn;
-  }
   auto launch_router = [&]() -> cudaError_t {
     cudaError_t err = mark(0, sm);
     if (err != cudaSuccess) return err;
     err = launch(pick_router(s.n_experts), ra.G, router_threads_for(s.n_experts),
-                 moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra, *h->tab13);
+                 moe::router_smem_bytes(batch, s.n_experts, h->router_chunk_rows), sm, true, ra);
     if (err != cudaSuccess) return err;
     ++kernels;
     return mark(1, sm);
   };
 
+  // the combine kernel also counts the stages of this forward's units per
+  // token class (from the plan the expert kernels consumed)
+  moe::StageCountArgs sc{};
+  sc.plan = h->at<Plan>(h->L.plan);
+  sc.counts = h->at<unsigned long long>(h->L.stage_counts);
+  sc.n_su = n_su;
+  sc.batch = batch;
+  sc.H = s.hidden;
+  sc.I = s.inter;
+  sc.Is = s.n_shared ? s.shared_inter : 0;
+  sc.kc = h->use_tc ? moe::kNumClasses - 1 : kc;
+  sc.max_units = (int)max_units(&s);
+  sc.fp8 = f8 ? 1 : 0;
   auto launch_combine = [&](bool pdl) -> cudaError_t {
     const int nvec = batch * s.hidden / 8;
     cudaError_t err = launch(moe::combine_residual_kernel, ceil_div(nvec, 256), 256, 0, sm, pdl,
-                             static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec);
+                             static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec,
+                             sc);
     if (err != cudaSuccess) return err;
     ++kernels;
     return mark(3, sm);
   };
 
   if (!two_stream) {
-    // ------------------------- default: router + expert kernel (+ combine)
+    // -------------------------------------------- default: three kernels
     MmaArgs ma = base;
     ma.n_su = n_su;
     ma.has_routed = 1;
-    if (fused_combine) {
-      ma.out = static_cast<__nv_bfloat16*>(out);
-      ma.cb_cnt = h->at<unsigned>(h->L.cb_cnt);
-    }
     if ((e = launch_router()) != cudaSuccess) return bail(e);
     if ((e = mark(4, sm)) != cudaSuccess) return bail(e);
     e = launch(mlp, h->grid_routed, mlp_threads, smem, sm, true, ma, *h->tab13, *h->tab2);
     if (e != cudaSuccess) return bail(e);
     ++kernels;
     if ((e = mark(2, sm)) != cudaSuccess || (e = mark(5, sm)) != cudaSuccess) return bail(e);
-    if (fused_combine) {
-      if ((e = mark(3, sm)) != cudaSuccess) return bail(e);
-    } else if ((e = launch_combine(true)) != cudaSuccess) {
-      return bail(e);
-    }
+    if ((e = launch_combine(true)) != cudaSuccess) return bail(e);
   } else {
     // ------------------------------------ MOE_FLAG_TWO_STREAM: four kernels
     // Shared expert (weight 1, all tokens): on stream_aux, forked after the
@@ -657,7 +706,8 @@ int wait_for_handle_work(moe_decode_ctx* h) {
 
 int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, const void* const* w13,
                     const void* const* w2, const void* shared_w13, const void* shared_w2, void* out,
-                    int32_t* topk_ids, float* topk_w, int batch, cudaStream_t sm, cudaStream_t sa);
+                    int32_t* topk_ids, float* topk_w, int batch, cudaStream_t sm, cudaStream_t sa,
+                    const Fp8Scales* f8);
 int refresh_maps(moe_decode_ctx* h, const void* const* w13, const void* const* w2, const void* sw13,
                  const void* sw2, cudaStream_t sm);
 
@@ -685,6 +735,9 @@ int forward_host_graph(moe_decode_ctx* h, const void* x_host, const void* router
     h->dirty = false;
   }
   if (!h->host_exec || batch != h->host_key_batch || key != h->host_key) {
+    // the legacy default stream cannot be captured; nor can a stream that is
+    // already being captured
+    if (sm == nullptr || sm == cudaStreamLegacy) return MOE_ERR_UNSUPPORTED_SHAPE;
     cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(sm, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) {
       cudaGetLastError();
@@ -694,7 +747,10 @@ int forward_host_graph(moe_decode_ctx* h, const void* x_host, const void* router
       const int rc = refresh_maps(h, w13, w2, sw13, sw2, sm);
       if (rc != MOE_OK) return rc;
     }
-    if ((e = cudaStreamBeginCapture(sm, cudaStreamCaptureModeThreadLocal)) != cudaSuccess) return fail_cuda(e);
+    if (cudaStreamBeginCapture(sm, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_UNSUPPORTED_SHAPE;
+    }
     const size_t xb = (size_t)batch * h->s.hidden * 2;
     int rc = MOE_OK;
     e = cudaMemcpyAsync(h->ws + h->L.x_stage, x_host, xb, cudaMemcpyHostToDevice, sm);
@@ -702,7 +758,7 @@ int forward_host_graph(moe_decode_ctx* h, const void* x_host, const void* router
     const uint64_t fw = h->stats.forwards, kl = h->stats.kernels_launched;
     if (rc == MOE_OK)
       rc = enqueue_forward(h, h->ws + h->L.x_stage, router_w, w13, w2, sw13, sw2, out_d,
-                           static_cast<int32_t*>(ids_d), static_cast<float*>(w_d), batch, sm, sa);
+                           static_cast<int32_t*>(ids_d), static_cast<float*>(w_d), batch, sm, sa, nullptr);
     h->stats.forwards = fw;  // counted below, once per launch
     h->stats.kernels_launched = kl;
     cudaGraph_t g = nullptr;
@@ -853,7 +909,6 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
   ra.topk_ids = topk_ids;
   ra.topk_w = topk_w;
   ra.spin_limit = moe::kSpinLimit;
-  ra.prefetch_stages = 0;  // no expert kernel follows
   const size_t smem = moe::router_smem_bytes(batch, n_experts, ra.chunk_rows);
   cudaFuncAttributes fa{};
   const RouterKernel rk = pick_router(n_experts);
@@ -862,8 +917,7 @@ int moe_router_topk_noalloc(const void* x, const void* router_w, const float* ro
     e = cudaFuncSetAttribute(rk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return fail_cuda(e);
   }
-  static const ExpertTable no_experts{};  // not read: prefetch is off
-  e = launch(rk, ra.G, router_threads_for(n_experts), smem, st, false, ra, no_experts);
+  e = launch(rk, ra.G, router_threads_for(n_experts), smem, st, false, ra);
   if (e != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
 }
@@ -925,11 +979,10 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
   h->grid_routed_auto = h->grid_routed == 0;
   if (h->grid_routed == 0) h->grid_routed = h->num_sms;
   h->grid_shared = env_int("MOE_DECODE_GRID_SHARED", 0, 0, 8 * h->num_sms);  // 0: sized per call
-  h->prefetch_stages = env_int("MOE_DECODE_PREFETCH_STAGES", 0, 0, moe::kMaxChunk);
-  h->lookahead = env_int("MOE_DECODE_LOOKAHEAD", 0, 0, 64);
   h->host_graph_on = env_int("MOE_DECODE_HOST_GRAPH", 1, 0, 1) == 1;
+  h->stagger = env_int("MOE_DECODE_STAGGER", 8, 0, moe::kMaxChunk);
   {
-    int gr = h->num_sms;
+    int gr = env_int("MOE_DECODE_ROUTER_CTAS", h->num_sms, 1, h->num_sms);
     const int cap = shapes->hidden / 8;
     h->grid_router_max = gr < cap ? gr : cap;
     if (h->grid_router_max < 1) h->grid_router_max = 1;
@@ -974,9 +1027,9 @@ int moe_decode_init(const moe_decode_shapes* shapes, moe_decode_t* out_handle) {
                   encode_matrix_map(probe, h->ws, shapes->hidden, 2 * shapes->inter);
     h->use_tc = h->use_tmap && (shapes->flags & MOE_FLAG_TCGEN05) != 0;
     if (h->use_tmap) {
-      h->map_ptrs.assign(2 * (size_t)shapes->n_experts + 2, nullptr);
-      e = cudaMallocHost(reinterpret_cast<void**>(&h->maps_host),
-                         (2 * (size_t)shapes->n_experts + 2) * moe::kTensorMapBytes);
+      const size_t nm = 2 * (size_t)shapes->n_experts + 2;
+      h->map_ptrs.assign(nm, nullptr);
+      e = cudaMallocHost(reinterpret_cast<void**>(&h->maps_host), nm * moe::kTensorMapBytes);
       if (e != cudaSuccess) rc = fail_cuda(e);
     }
   }
@@ -997,14 +1050,37 @@ int moe_decode_forward(moe_decode_t h, const void* x, const void* router_w, cons
   if (batch == 0) return MOE_OK;
   DeviceGuard guard(h->device);
   if (!guard.ok) return fail_cuda(cudaGetLastError());
+  if (h->s.flags & MOE_FLAG_FP8_WEIGHTS) return MOE_ERR_INVALID_ARG;  // moe_decode_forward_fp8
   return enqueue_forward(h, x, router_w, w13, w2, shared_w13, shared_w2, out, topk_ids, topk_w, batch,
-                         static_cast<cudaStream_t>(stream_main), static_cast<cudaStream_t>(stream_aux));
+                         static_cast<cudaStream_t>(stream_main), static_cast<cudaStream_t>(stream_aux), nullptr);
+}
+
+int moe_decode_forward_fp8(moe_decode_t h, const void* x, const void* router_w, const void* const* w13q,
+                           const void* const* w13s, const void* const* w2q, const void* const* w2s,
+                           const void* shared_w13q, const void* shared_w13s, const void* shared_w2q,
+                           const void* shared_w2s, void* out, int32_t* topk_ids, float* topk_w, int32_t batch,
+                           void* stream_main, void* stream_aux) {
+  if (!h || !(h->s.flags & MOE_FLAG_FP8_WEIGHTS) || !h->use_tmap) return MOE_ERR_INVALID_ARG;
+  int rc = check_forward_args(h, x, router_w, w13q, w2q, shared_w13q, shared_w2q, out, topk_ids, topk_w, batch, true);
+  if (rc != MOE_OK) return rc;
+  if (batch == 0) return MOE_OK;
+  if (!w13s || !w2s) return MOE_ERR_INVALID_ARG;
+  for (int i = 0; i < h->s.n_experts; ++i)
+    if (!w13s[i] || !w2s[i] || !aligned16(w13s[i]) || !aligned16(w2s[i])) return MOE_ERR_INVALID_ARG;
+  if (h->s.n_shared && (!shared_w13s || !shared_w2s || !aligned16(shared_w13s) || !aligned16(shared_w2s)))
+    return MOE_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return fail_cuda(cudaGetLastError());
+  const Fp8Scales f8{w13s, w2s, shared_w13s, shared_w2s};
+  return enqueue_forward(h, x, router_w, w13q, w2q, shared_w13q, shared_w2q, out, topk_ids, topk_w, batch,
+                         static_cast<cudaStream_t>(stream_main), static_cast<cudaStream_t>(stream_aux), &f8);
 }
 
 int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* router_w, const void* const* w13,
                             const void* const* w2, const void* shared_w13, const void* shared_w2,
                             void* out_host, int32_t* ids_host, float* w_host, int32_t batch, void* stream_main,
                             void* stream_aux) {
+  if (h && (h->s.flags & MOE_FLAG_FP8_WEIGHTS)) return MOE_ERR_INVALID_ARG;  // bf16 weights only
   int rc = check_forward_args(h, x_host, router_w, w13, w2, shared_w13, shared_w2, out_host, ids_host, w_host,
                               batch, false);
   if (rc != MOE_OK) return rc;
@@ -1038,7 +1114,7 @@ int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* rout
   if ((e = cudaMemcpyAsync(xd, x_host, xb, cudaMemcpyHostToDevice, sm)) != cudaSuccess) return fail_cuda(e);
   rc = enqueue_forward(h, xd, router_w, w13, w2, shared_w13, shared_w2, direct ? od_m : od,
                        static_cast<int32_t*>(direct ? idd_m : idd), static_cast<float*>(direct ? wd_m : wd), batch,
-                       sm, static_cast<cudaStream_t>(stream_aux));
+                       sm, static_cast<cudaStream_t>(stream_aux), nullptr);
   if (rc != MOE_OK) return rc;
   if (!direct) {
     if ((e = cudaMemcpyAsync(out_host, od, xb, cudaMemcpyDeviceToHost, sm)) != cudaSuccess) return fail_cuda(e);

@@ -346,7 +346,8 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
     const float* lg = s_lg + (size_t)(t - tb0) * E;
     float v[NV];
     uint32_t taken = 0;
-    if (k > 8) {
+    const bool rounds = k > 8;
+    if (rounds) {
 #pragma unroll
       for (int i = 0; i < NV; ++i) {
         const int e = lane + 32 * i;
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
     };
     int my_id = -1;
     float my_v = -INFINITY;
-    if (k <= 8) {
+    if (!rounds) {
       float tv[8];
       int ti[8];
       warp_top8(lg, s_bias, E, lane, tv, ti);

@@ -173,3 +173,69 @@ def make_router(shape: BlockShape, seed: int = 0, routing: str = "uniform"):
     router_w = _normal_bf16((shape.hidden, shape.n_experts), WEIGHT_STD, seed_for(seed, "router_w"), "cpu")
     bias = zipf_log_prior(shape.n_experts, seed, "cpu") if routing == "zipf" else None
     return router_w, bias
+
+
+@dataclasses.dataclass
+class Fp8BlockWeights:
+    """Expert weights as e4m3 codes with fp32 block scales (the layout the
+    library's fp8 entry point takes): q13 [E, 2I, H] and q2 [E, H, I] uint8
+    ([out, in]); s13 [E, ceil(H/128), P13] and s2 [E, ceil(I/128), P2]
+    float32, scale[i/128, o/128] of output o and input i, rows padded to a
+    multiple of 4 floats; the shared expert's likewise without the E axis."""
+    router_w: torch.Tensor
+    q13: torch.Tensor
+    s13: torch.Tensor
+    q2: torch.Tensor
+    s2: torch.Tensor
+    shared_q13: Optional[torch.Tensor]
+    shared_s13: Optional[torch.Tensor]
+    shared_q2: Optional[torch.Tensor]
+    shared_s2: Optional[torch.Tensor]
+    router_bias: Optional[torch.Tensor]
+
+
+def scale_pitch(outs: int) -> int:
+    """Floats per row of an e4m3 matrix's block scales (padded to 16 bytes)."""
+    return -(-(-(-outs // 128)) // 4) * 4
+
+
+def _fp8_matrix(outs: int, ins: int, std: float, seed: int, device):
+    """One [outs, ins] matrix ~ N(0, std) drawn in fp32 and stored as e4m3
+    codes with one fp32 scale per 128 x 128 block (scale = block absmax / 448,
+    so the block's largest magnitude maps to e4m3's largest finite value)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    w = torch.randn(outs, ins, generator=g, device=device, dtype=torch.float32).mul_(std)
+    ob, ib = -(-outs // 128), -(-ins // 128)
+    wp = torch.zeros(ob * 128, ib * 128, device=device, dtype=torch.float32)
+    wp[:outs, :ins] = w
+    blocks = wp.view(ob, 128, ib, 128)
+    amax = blocks.abs().amax(dim=(1, 3))                       # [ob, ib]
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (blocks / scale[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    q = q.reshape(ob * 128, ib * 128)[:outs, :ins].contiguous()
+    s = torch.zeros(ib, scale_pitch(outs), device=device, dtype=torch.float32)
+    s[:, :ob] = scale.t()
+    return q, s
+
+
+def make_fp8_weights(shape: BlockShape, seed: int = 0, device="cpu", routing: str = "uniform",
+                     router_device=None) -> Fp8BlockWeights:
+    """A block with e4m3 expert weights (routed and shared) and bf16 router
+    weights, each matrix from its own sub-seed (different from make_weights')."""
+    H, E, I, Is = shape.hidden, shape.n_experts, shape.inter, shape.shared_inter
+    rdev = device if router_device is None else router_device
+    router_w = _normal_bf16((H, E), WEIGHT_STD, seed_for(seed, "router_w"), rdev).to(device)
+    q13 = torch.empty(E, 2 * I, H, dtype=torch.uint8, device=device)
+    s13 = torch.empty(E, -(-H // 128), scale_pitch(2 * I), dtype=torch.float32, device=device)
+    q2 = torch.empty(E, H, I, dtype=torch.uint8, device=device)
+    s2 = torch.empty(E, -(-I // 128), scale_pitch(H), dtype=torch.float32, device=device)
+    for e in range(E):
+        q13[e], s13[e] = _fp8_matrix(2 * I, H, WEIGHT_STD, seed_for(seed, "fp8_w13", e), device)
+        q2[e], s2[e] = _fp8_matrix(H, I, WEIGHT_STD, seed_for(seed, "fp8_w2", e), device)
+    sq13 = ss13 = sq2 = ss2 = None
+    if shape.n_shared:
+        sq13, ss13 = _fp8_matrix(2 * Is, H, WEIGHT_STD, seed_for(seed, "fp8_shared_w13"), device)
+        sq2, ss2 = _fp8_matrix(H, Is, WEIGHT_STD, seed_for(seed, "fp8_shared_w2"), device)
+    bias = zipf_log_prior(E, seed, device) if routing == "zipf" else None
+    return Fp8BlockWeights(router_w, q13, s13, q2, s2, sq13, ss13, sq2, ss2, bias)

@@ -47,12 +47,11 @@ class Run:
                              two_stream=two_stream, tcgen05=tcgen05, extra_flags=extra_flags)
 
     def kernels_per_forward(self):
-        """Kernels one forward enqueues: router and expert kernel (which ends
-        with the combine) by default, plus a combine kernel on tcgen05;
+        """Kernels one forward enqueues: router, expert kernel, combine by default;
         router, routed experts, [shared expert], combine with two streams."""
         if self.blk.two_stream:
             return 4 if self.s.n_shared else 3
-        return 3 if self.blk.tcgen05 else 2
+        return 3
 
     def forward(self, x, stream_aux=None, w13=None, w2=None):
         B = x.shape[0]
@@ -71,6 +70,7 @@ class Run:
 # 64 KB weight stage), restated to predict the device-side stage counters.
 CLASS_LW = (2048, 1024, 512)
 CLASS_ROWS = (16, 32, 64)
+CLASS_ROWS_FP8 = (32, 64, 64)  # stages of e4m3 weights
 UNIT_TOKENS = 32
 
 
@@ -78,24 +78,17 @@ def token_class(n):
     return 0 if n <= 8 else (1 if n <= 16 else 2)
 
 
-def unit_stages(c, up, H, I):
-    """Stages of a unit's UP or DOWN list.  UP: panels of lw/2 gate (+ up)
-    columns, r-row stages.  DOWN: full panels of lw columns, then a ragged
-    last panel (H mod lw columns) in the next class's geometry when it fits
-    that width."""
-    lw, r = CLASS_LW[c], CLASS_ROWS[c]
+def unit_stages(c, up, H, I, fp8=False):
+    """Stages of a unit's UP list (panels of lw/2 gate + up columns, r-row
+    stages) or DOWN list (panels of lw columns, r-row stages)."""
+    lw, r = CLASS_LW[c], (CLASS_ROWS_FP8 if fp8 else CLASS_ROWS)[c]
     cdiv = lambda a, b: -(-a // b)
     if up:
         return cdiv(I, lw // 2) * cdiv(H, r)
-    full = (H // lw) * cdiv(I, r)
-    rem = H % lw
-    if rem == 0:
-        return full
-    g = c + 1 if c + 1 < len(CLASS_LW) and CLASS_LW[c + 1] >= rem else c
-    return full + cdiv(I, CLASS_ROWS[g])
+    return cdiv(H, lw) * cdiv(I, r)
 
 
-def expected_stages(shape, ids, batch):
+def expected_stages(shape, ids, batch, fp8=False):
     """(up[3], down[3]) stages one forward streams per token class: the shared
     expert in units of up to 32 tokens, each selected expert in units of up to
     32 of the tokens that chose it."""
@@ -108,8 +101,8 @@ def expected_stages(shape, ids, batch):
         units += [(min(UNIT_TOKENS, int(n) - u), shape.inter) for u in range(0, int(n), UNIT_TOKENS)]
     for n, I in units:
         c = token_class(n)
-        up[c] += unit_stages(c, True, shape.hidden, I)
-        down[c] += unit_stages(c, False, shape.hidden, I)
+        up[c] += unit_stages(c, True, shape.hidden, I, fp8)
+        down[c] += unit_stages(c, False, shape.hidden, I, fp8)
     return up, down
 
 

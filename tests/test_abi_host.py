@@ -65,7 +65,8 @@ def test_workspace_bytes_and_shape_validation(lib):
     assert 0 < tiny < full
     bad = [dict(hidden=7170), dict(hidden=0), dict(n_experts=12), dict(n_experts=2048), dict(top_k=0),
            dict(top_k=33), dict(top_k=9, n_experts=8), dict(inter=100), dict(n_shared=2),
-           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=8), dict(flags=9), dict(flags=1 << 31)]
+           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=16), dict(flags=17), dict(flags=1 << 31),
+           dict(flags=8, hidden=7168 + 64), dict(flags=8, inter=2048 + 64), dict(flags=8 | 2)]
     for kw in bad:
         sh = _shapes(**kw)
         assert lib.moe_decode_workspace_bytes(ctypes.byref(sh)) == 0, kw
@@ -76,6 +77,8 @@ def test_workspace_bytes_and_shape_validation(lib):
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TWO_STREAM))) == full
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TCGEN05))) == full
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=3))) == full
+    # e4m3 expert weights: whole 128 x 128 scale blocks, not with tcgen05
+    assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_FP8_WEIGHTS))) == full
     # the testing-only hold flag is accepted too (the handle's first forward
     # withholds one panel publication)
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TEST_HOLD_PANEL))) == full
@@ -93,6 +96,7 @@ def test_null_arguments_are_rejected_on_the_host(lib):
     assert lib.moe_decode_forward(None, *([None] * 9), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_forward_host(None, *([None] * 9), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_set_wait_limit(None, 100) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_forward_fp8(None, *([None] * 13), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
 
 
 def test_init_without_a_gpu_reports_no_device(lib):

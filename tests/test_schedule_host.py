@@ -8,6 +8,8 @@ kernel runs.  Properties, for many stage counts T and grid sizes G:
   * make_sched's chunks hold at most kMaxChunk stages, and its tail of
     one-stage tickets stays bounded (about 2G, whatever T is);
   * make_round hands out whole-grid rounds: a chunk size of max(T / G, 1).
+  * with staggered starts, the first G big chunks are c_big - (tk mod stag)
+    stages, never under half a big chunk, and the tiling properties hold.
 A lost stage would drop part of a weight matrix from the sums; a repeated one
 would count it twice.
 """
@@ -47,10 +49,21 @@ static void walk(const Sched& s, int T, int G, int max_chunk, int* bad) {
 // remainder (smaller than one quarter chunk)
 static void check_bands(const Sched& s, int T, int G, int* bad) {
   const int tail = s.n_tickets - s.n_big - s.n_mid;
+  const int taken = sched_stagger_sum(std::min(s.n_big, G), s.stag);
   if (tail != T - s.T2) *bad = fail("tail tickets", T, G);
   if (tail > std::min(T, 2 * G) + s.c_mid - 1) *bad = fail("tail length", T, G);
-  if (s.n_mid > 3 * G + s.c_big / s.c_mid + 1) *bad = fail("quarter band", T, G);
+  if (s.n_mid > 3 * G + s.c_big / s.c_mid + 1 + taken / s.c_mid) *bad = fail("quarter band", T, G);
   if (s.c_mid != std::max(s.c_big / 4, 1)) *bad = fail("quarter size", T, G);
+  if (s.stag > 1 && s.stag > s.c_big / 2) *bad = fail("stagger bound", T, G);
+}
+// staggered starts: the first G big chunks have c_big - (tk mod stag) stages
+static void check_stagger(const Sched& s, int T, int G, int* bad) {
+  for (int tk = 0; tk < std::min(s.n_big, G); ++tk) {
+    int b, e;
+    sched_range(s, tk, b, e);
+    const int want = s.c_big - (s.stag > 1 ? tk %% s.stag : 0);
+    if (e - b != want || e - b < (s.c_big + 1) / 2) { *bad = fail("staggered chunk", T, G); return; }
+  }
 }
 int main() {
   const int grids[] = {1, 2, 3, 7, 64, 74, 148, 296};
@@ -63,6 +76,12 @@ int main() {
       const Sched b = make_sched(T, G, 4);
       walk(b, T, G, kMaxChunk, &bad);
       check_bands(b, T, G, &bad);
+      for (int stag : {4, 8, 13}) {
+        const Sched c = make_sched(T, G, 4, stag);
+        walk(c, T, G, kMaxChunk, &bad);
+        check_bands(c, T, G, &bad);
+        check_stagger(c, T, G, &bad);
+      }
     }
     const int big[] = {20000, 131071, 390000, 524287};
     for (int T : big) {
@@ -70,6 +89,12 @@ int main() {
       const Sched b = make_sched(T, G, 4);
       walk(b, T, G, kMaxChunk, &bad);
       check_bands(b, T, G, &bad);
+      for (int stag : {4, 8, 13}) {
+        const Sched c = make_sched(T, G, 4, stag);
+        walk(c, T, G, kMaxChunk, &bad);
+        check_bands(c, T, G, &bad);
+        check_stagger(c, T, G, &bad);
+      }
     }
   }
   if (!bad) std::printf("ok\n");
