@@ -97,20 +97,29 @@ __host__ __device__ constexpr int class_rows(int c) { return c == 0 ? 16 : (c ==
 __host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : 4); }
 // class of a unit with n <= kUnitTok tokens
 __host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : 2); }
-// FP8 (e4m3) weights: the same panel widths, stages of 32 rows (class 0,
-// 2048 x 32 = 64 KB) and 64 rows (classes 1 and 2: 64 KB and 32 KB), so the
-// accumulators per consumer warp are the same as for bf16 weights and the
-// tokens' activation rows fit the same buffer.
-__host__ __device__ constexpr int class_rows_fp8(int c) { return c == 0 ? 32 : 64; }
-__host__ __device__ constexpr int geo_rows(int c, bool fp8) { return fp8 ? class_rows_fp8(c) : class_rows(c); }
-// Bytes of the fp8 weights of a stage (the block scales follow them).
-constexpr int kFp8StageWBytes = 65536;
+// FP8 (e4m3) weights, stored [out, in]: a stage is 128 input rows -- one
+// 128-byte line of every weight row it touches, and exactly one block of the
+// 128 x 128 block scales along the input -- by 512 columns (classes 0 and 1,
+// 64 KB) or 256 columns (class 2, 32 KB, so the 32 tokens' 128-row
+// activations still fit the stage).  Whole lines keep DRAM and L2 reading
+// each weight byte once; narrower K slices of a row (32 bytes per stage) made
+// the TMA fetch every line twice.
+constexpr int kFp8Rows = 128;
+__host__ __device__ constexpr int class_lw_fp8(int c) { return c == 2 ? 256 : 512; }
+__host__ __device__ constexpr int geo_rows(int c, bool fp8) { return fp8 ? kFp8Rows : class_rows(c); }
+__host__ __device__ constexpr int geo_lw(int c, bool fp8) { return fp8 ? class_lw_fp8(c) : class_lw(c); }
+// Bytes of a class's fp8 weights in a stage; the stage's row of block scales
+// follows them, and the tokens' activations start 1 KB after that.
+__host__ __device__ constexpr int fp8_stage_wbytes(int c) { return class_lw_fp8(c) * kFp8Rows; }
+__host__ __device__ constexpr int fp8_stage_xoff(int c) { return fp8_stage_wbytes(c) + 1024; }
+constexpr int kFp8XPitch = kFp8Rows * 2 + 16;  // bytes per token row of activations
 // Consumer warps: sixteen in every instance (seventeen warps with the
 // producer cap a thread at 96 registers, room for the 32 accumulators).
 __host__ __device__ constexpr int consumer_warps_for(int) { return 16; }
 __host__ __device__ constexpr int expert_threads(int kc) { return (consumer_warps_for(kc) + 1) * 32; }
 // m-tiles (16 columns) per consumer warp for class c with cw consumer warps
 __host__ __device__ constexpr int class_mt(int c, int cw) { return class_lw(c) / (cw * 16); }
+__host__ __device__ constexpr int geo_mt(int c, int cw, bool fp8) { return geo_lw(c, fp8) / (cw * 16); }
 // accumulator fragments (of 4 floats) a consumer thread needs for classes <= KC
 __host__ __device__ constexpr int acc_frags(int kc) { return class_mt(0, consumer_warps_for(kc)) * class_nt(0); }
 static_assert(class_mt(1, 16) * class_nt(1) == acc_frags(1) && class_mt(2, 16) * class_nt(2) == acc_frags(2),
@@ -123,6 +132,14 @@ constexpr int kStageWBytes = cmax(stage_w_bytes(0), cmax(stage_w_bytes(1), stage
 constexpr int kStageXBytes = kUnitTok * (class_rows(2) * 2 + 16);                                 // 4608
 constexpr int kStageBytesMma = (kStageWBytes + kStageXBytes + 1023) / 1024 * 1024;               // 70 KB
 static_assert(kStageBytesMma % 1024 == 0, "128-byte swizzle atoms need 1 KB aligned stages");
+static_assert(fp8_stage_xoff(0) + 8 * kFp8XPitch <= kStageBytesMma &&
+                  fp8_stage_xoff(1) + 16 * kFp8XPitch <= kStageBytesMma &&
+                  fp8_stage_xoff(2) + 32 * kFp8XPitch <= kStageBytesMma,
+              "fp8 stages: weights, scale row and the class's token rows fit one stage");
+static_assert(geo_mt(0, 16, true) * class_nt(0) <= class_mt(0, 16) * class_nt(0) &&
+                  geo_mt(1, 16, true) * class_nt(1) <= class_mt(0, 16) * class_nt(0) &&
+                  geo_mt(2, 16, true) * class_nt(2) <= class_mt(0, 16) * class_nt(0),
+              "fp8 classes need no more accumulators than the bf16 ones");
 constexpr int kMaxStagesMma = 3;
 constexpr int kMaxChunk = 64;  // stages per queue grab, at most
 // tensor-map path: boxes of {64 columns, 16 rows, 4 column chunks}
@@ -132,8 +149,9 @@ constexpr int kBoxChunks = 4;
 constexpr int kChunkTile = kBoxRows * kChunkCols * 2;  // 2048 B: one chunk of one 16-row block
 constexpr int kBoxBytes = kChunkTile * kBoxChunks;     // 8192 B per load
 constexpr int kTensorMapBytes = 128;
-// UP panels of a unit, at most: ceil(I / 256) (class 2); sizes the panel counters
-__host__ __device__ inline int max_up_panels(int I) { return (I + class_lw(2) / 2 - 1) / (class_lw(2) / 2); }
+// UP panels of a unit, at most: ceil(I / 128) (fp8 class 2; bf16 class 2
+// needs ceil(I / 256)); sizes the panel counters
+__host__ __device__ inline int max_up_panels(int I) { return (I + class_lw_fp8(2) / 2 - 1) / (class_lw_fp8(2) / 2); }
 
 enum : int { kKindUp = 0, kKindDown = 1, kKindEnd = 2 };
 enum : int { kFirst = 1, kLast = 2 };
@@ -205,8 +223,8 @@ __host__ __device__ inline size_t mma_smem_bytes(int n_stages) {
 
 // Panels and stages per panel of one unit with class `cls`, UP or DOWN list
 // (I: the unit's intermediate size).
-__host__ __device__ __forceinline__ int unit_panels(int cls, bool up, int H, int I) {
-  const int lw = class_lw(cls);
+__host__ __device__ __forceinline__ int unit_panels(int cls, bool up, int H, int I, bool fp8 = false) {
+  const int lw = geo_lw(cls, fp8);
   return up ? (I + lw / 2 - 1) / (lw / 2) : (H + lw - 1) / lw;
 }
 __host__ __device__ __forceinline__ int unit_panel_stages(int cls, bool up, int H, int I, bool fp8 = false) {
@@ -214,7 +232,7 @@ __host__ __device__ __forceinline__ int unit_panel_stages(int cls, bool up, int 
   return up ? (H + r - 1) / r : (I + r - 1) / r;
 }
 __host__ __device__ __forceinline__ int unit_stages(int cls, bool up, int H, int I, bool fp8 = false) {
-  return unit_panels(cls, up, H, I) * unit_panel_stages(cls, up, H, I, fp8);
+  return unit_panels(cls, up, H, I, fp8) * unit_panel_stages(cls, up, H, I, fp8);
 }
 
 // Ticket schedule over a segment of T stages for a grid of G CTAs
@@ -415,43 +433,41 @@ __device__ __forceinline__ void mma_stage(float (&acc)[NF][4], uint32_t sw, uint
   }
 }
 
-// One stage of tensor-core work on e4m3 weights (class C geometry: LWc
-// columns x class_rows_fp8(C) rows), accumulated into the same fragments as
-// mma_stage.  The stage holds the weights as [32-row chunk][column][32 bytes
-// of rows] -- each column's rows contiguous, as the [out, in] layout stores
-// them -- with TMA's 32-byte swizzle (the 16-byte half of a 32-byte row is
-// XORed with bit 2 of the column index).  ldmatrix (b16, not transposed)
-// gives a lane (g, t) of an 8 x 8 tile the four bytes of rows 4t .. 4t+3 of
-// column g: converted to f16, its low pair is the A operand's first k pair
-// and its high pair the second, which is the k order (0 1 | 8 9 ...)
-// relabelled; the tokens' fragments are loaded in the same order (rows 4t ..
-// 4t+3 as b0, b1), so each product pairs the same row of both.  Every e4m3
-// value is exact in f16 and the activations (bf16, |v| well inside f16's
-// range) are converted to f16 too; the stage's partial products (fp32) are
-// multiplied by the warp's block scale -- all of a warp's columns and a
-// stage's rows lie in one 128 x 128 block -- and added to the accumulators.
+// One stage of tensor-core work on e4m3 weights (class C: class_lw_fp8(C)
+// columns x 128 rows), accumulated into the same fragments as mma_stage.
+// The stage holds the weights as [column][128 bytes of rows] -- each column's
+// rows contiguous, as the [out, in] layout stores them -- with TMA's 128-byte
+// swizzle (16-byte unit u of column c sits at unit u ^ (c % 8)).  ldmatrix
+// (b16, not transposed) gives a lane (g, t) of an 8 x 8 tile the four bytes
+// of rows 4t .. 4t+3 of column g: converted to f16, its low pair is the A
+// operand's first k pair and its high pair the second, which is the k order
+// (0 1 | 8 9 ...) relabelled; the tokens' fragments are loaded in the same
+// order (rows 4t .. 4t+3 as b0, b1), so each product pairs the same row of
+// both.  Every e4m3 value is exact in f16 and the activations (bf16, |v| well
+// inside f16's range) are converted to f16 too; each product (fp32) is
+// multiplied by the warp's block scale -- a warp's columns and a stage's
+// rows lie in one 128 x 128 block -- and added to the accumulators.
 template <int C, int NF, int CW>
 __device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, uint32_t sx, const float* srow,
                                               int LW, int nrows, int ntiles, bool up, int c0, int uoff, int I,
                                               int warp, int lane) {
-  constexpr int LWc = class_lw(C), R = class_rows_fp8(C);
-  constexpr int MT = class_mt(C, CW), NT = class_nt(C), KC32 = R / 32;
+  constexpr int MT = geo_mt(C, CW, true), NT = class_nt(C), KP = kFp8Rows / 32;
   static_assert(MT * NT <= NF, "accumulator budget");
-  constexpr int xpitch = R * 2 + 16;
+  constexpr int xpitch = kFp8XPitch;
   const int m0 = warp * MT * 16;
   if (m0 >= LW) return;
   const int out0 = up ? (m0 < uoff ? c0 + m0 : I + c0 + (m0 - uoff)) : c0 + m0;
   const float sc = srow[out0 >> 7];
   const int g = lane >> 2, tq = lane & 3;
   const int li = lane >> 3, lr = lane & 7;
-  // tokens' fragments of tile nt for this 32-row chunk: rows 4tq .. 4tq + 3
+  // tokens' fragments of tile nt for the 32-row slice kp: rows 4tq .. 4tq + 3
   // of each 16-row half, converted to f16 (zero past the stage's rows)
-  auto load_b = [&](int kc, int nt, uint32_t (&b)[4]) {
-    const uint32_t a = sx + (uint32_t)(nt * 8 + g) * xpitch + (uint32_t)(kc * 32 + 4 * tq) * 2;
+  auto load_b = [&](int kp, int nt, uint32_t (&b)[4]) {
+    const uint32_t a = sx + (uint32_t)(nt * 8 + g) * xpitch + (uint32_t)(kp * 32 + 4 * tq) * 2;
     uint32_t v0, v1, v2, v3;
     asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(a));
     asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v2), "=r"(v3) : "r"(a + 32));
-    const bool h0 = kc * 32 + 4 * tq < nrows, h1 = kc * 32 + 16 + 4 * tq < nrows;
+    const bool h0 = kp * 32 + 4 * tq < nrows, h1 = kp * 32 + 16 + 4 * tq < nrows;
     b[0] = h0 ? bf16x2_to_f16x2(v0) : 0u;
     b[1] = h0 ? bf16x2_to_f16x2(v1) : 0u;
     b[2] = h1 ? bf16x2_to_f16x2(v2) : 0u;
@@ -460,20 +476,20 @@ __device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, 
   // one token tile: its fragments stay in registers for all m-tiles; more
   // tiles: reloaded per m-tile (keeping them all costs spills)
   constexpr bool kKeepB = NT == 1;
-  // (the chunk loop stays rolled: unrolled, its hoisted addresses and
+  // (the slice loop stays rolled: unrolled, its hoisted addresses and
   // fragments spill in the classes with several token tiles)
 #pragma unroll 1
-  for (int kc = 0; kc < KC32; ++kc) {
-    if (kc * 32 >= nrows) break;
+  for (int kp = 0; kp < KP; ++kp) {
+    if (kp * 32 >= nrows) break;
     uint32_t bk[4] = {0u, 0u, 0u, 0u};
-    if (kKeepB) load_b(kc, 0, bk);
+    if (kKeepB) load_b(kp, 0, bk);
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       if (m0 + mt * 16 < LW) {
-        const int col = m0 + mt * 16 + (li & 1) * 8 + lr;   // local column of this lane's ldmatrix row
-        const int half = (li >> 1) ^ ((col >> 2) & 1);       // 32-byte swizzle
+        const int col = m0 + mt * 16 + (li & 1) * 8 + lr;  // local column of this lane's ldmatrix row
+        const int unit = (2 * kp + (li >> 1)) ^ (col & 7);   // 128-byte swizzle
         uint32_t r0, r1, r2, r3;
-        ldsm_x4(sw + (uint32_t)(kc * LWc * 32 + col * 32 + half * 16), r0, r1, r2, r3);
+        ldsm_x4(sw + (uint32_t)(col * 128 + unit * 16), r0, r1, r2, r3);
         if (kKeepB) {
           float t[4] = {0.f, 0.f, 0.f, 0.f};
           mma_f16_16816(t, e4m3x2_lo_to_f16x2(r0), e4m3x2_lo_to_f16x2(r1), e4m3x2_hi_to_f16x2(r0),
@@ -489,11 +505,11 @@ __device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, 
             const uint32_t ra = hf ? r2 : r0, rb = hf ? r3 : r1;
             const uint32_t a0 = e4m3x2_lo_to_f16x2(ra), a1 = e4m3x2_lo_to_f16x2(rb);
             const uint32_t a2 = e4m3x2_hi_to_f16x2(ra), a3 = e4m3x2_hi_to_f16x2(rb);
-            const bool live = kc * 32 + hf * 16 + 4 * tq < nrows;
+            const bool live = kp * 32 + hf * 16 + 4 * tq < nrows;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               if (nt < ntiles) {
-                const uint32_t ad = sx + (uint32_t)(nt * 8 + g) * xpitch + (uint32_t)(kc * 32 + hf * 16 + 4 * tq) * 2;
+                const uint32_t ad = sx + (uint32_t)(nt * 8 + g) * xpitch + (uint32_t)(kp * 32 + hf * 16 + 4 * tq) * 2;
                 uint32_t v0, v1;
                 asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v0), "=r"(v1) : "r"(ad));
                 float t[4] = {0.f, 0.f, 0.f, 0.f};
@@ -530,11 +546,11 @@ __device__ __forceinline__ int local_to_col(int l, bool up, int c0, int w, int u
 // reductions per lane of one quad.  (Gathering runs of 4 columns into one
 // lane with shuffles for vector reductions measured slower: the shuffles
 // cost more issue slots than the reductions they save.)
-template <int C, int NF, int CW>
+template <int C, int NF, int CW, bool FP8 = false>
 __device__ __forceinline__ void flush_piece(const float (&acc)[NF][4], float* base, size_t ld, int my_row,
                                             float my_wt, int ntok, bool up, int c0, int w, int uoff, int LW, int I,
                                             int warp, int lane) {
-  constexpr int MT = class_mt(C, CW), NT = class_nt(C);
+  constexpr int MT = geo_mt(C, CW, FP8), NT = class_nt(C);
   const int m0 = warp * MT * 16;
   if (m0 >= LW) return;
   const int gid = lane >> 2, tig = lane & 3;
@@ -777,7 +793,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
             }
           }
           u_cls = cls_of(u_ntok);
-          u_lw = class_lw(u_cls);
+          u_lw = geo_lw(u_cls, FP8);
           u_R = geo_rows(u_cls, FP8);
           u_S = unit_panel_stages(u_cls, up, H, u_I, FP8);
         }
@@ -835,20 +851,20 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         const int c0 = cp * (up ? lw / 2 : lw);
         const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);  // columns per half (UP) or panel (DOWN)
         const uint32_t wbytes = (uint32_t)w * 2;
-        const uint32_t pitch = (uint32_t)lw * 2 + 16, xpitch = (uint32_t)R * 2 + 16;
+        const uint32_t pitch = (uint32_t)lw * 2 + 16, xpitch = FP8 ? (uint32_t)kFp8XPitch : (uint32_t)R * 2 + 16;
         // tensor-map path: loads = halves x 16-row blocks x groups of 4 chunks
         const int t_ncg = (w / kChunkCols + kBoxChunks - 1) / kBoxChunks;
         const int t_nrb = R / kBoxRows;
-        // FP8: loads = halves x 256-column blocks x 32-row chunks, plus the
-        // stage's row of block scales (pitch floats per 128 weight rows)
-        const int f_nmb = (w + 255) / 256, f_per_half = f_nmb * (R / 32);
+        // FP8: loads = halves x 128-column boxes (each 128 rows x 128 bytes),
+        // plus the stage's row of block scales (pitch floats per 128 weight rows)
+        const int f_nb = (w + 127) / 128;
         const int f_pitch = up ? (seg == 0 ? args.sc_pitch13_s : args.sc_pitch13) : args.sc_pitch2;
-        const int t_nops = FP8 ? (up ? 2 : 1) * f_per_half : (up ? 2 : 1) * t_nrb * t_ncg;
-        const uint32_t wtotal = FP8 ? (uint32_t)t_nops * kBoxBytes + (uint32_t)f_pitch * 4u
+        const int t_nops = FP8 ? (up ? 2 : 1) * f_nb : (up ? 2 : 1) * t_nrb * t_ncg;
+        const uint32_t wtotal = FP8 ? (uint32_t)t_nops * (128u * kFp8Rows) + (uint32_t)f_pitch * 4u
                                     : (TMAP ? (uint32_t)t_nops * kBoxBytes : (uint32_t)nrows * (up ? 2u : 1u) * wbytes);
         const uint32_t bytes = wtotal + (uint32_t)ntok * nrows * 2;
         uint8_t* sw = stages + (size_t)slot * kStageBytesMma;
-        uint8_t* sx = sw + kStageWBytes;
+        uint8_t* sx = sw + (FP8 ? fp8_stage_xoff(cls) : kStageWBytes);
         StageHdr& hd = hdr[slot];
         if (lane < ntok) {
           hd.row[lane] = u_dst;
@@ -873,17 +889,17 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
         const void* act = up ? (const void*)(args.x + (size_t)u_src * H + row0)
                              : (const void*)((seg == 0 ? args.a_s : args.a) + (size_t)u_src * Iu + row0);
         if constexpr (FP8) {
-          // [32-row chunk][column][32 bytes] with 32-byte swizzle, UP's up
-          // half from local column lw / 2 (the weights are [out, in])
+          // [column][128 bytes of rows] with 128-byte swizzle, UP's up half
+          // from local column lw / 2 (the weights are [out, in]); the input
+          // coordinate row0 is a multiple of 128 bytes
           for (int o = lane; o < t_nops; o += 32) {
-            const int hh = o / f_per_half, rem = o - hh * f_per_half;
-            const int kc = rem / f_nmb, mb = rem - kc * f_nmb;
-            uint8_t* dst = sw + (size_t)kc * lw * 32 + (size_t)(hh * (lw / 2) + mb * 256) * 32;
-            const int m = (up ? (hh ? Iu + c0 : c0) : c0) + mb * 256;
-            tma_load_2d(dst, u_map, row0 + kc * 32, m, &full[slot], pol);
+            const int hh = o / f_nb, mb = o - hh * f_nb;
+            uint8_t* dst = sw + (size_t)(hh * (lw / 2) + mb * 128) * kFp8Rows;
+            const int m = (up ? (hh ? Iu + c0 : c0) : c0) + mb * 128;
+            tma_load_2d(dst, u_map, row0, m, &full[slot], pol);
           }
           if (lane == 31)  // u_W holds the matrix's scale array here
-            bulk_copy_g2s(sw + kFp8StageWBytes, reinterpret_cast<const float*>(u_W) + (size_t)(row0 >> 7) * f_pitch,
+            bulk_copy_g2s(sw + fp8_stage_wbytes(cls), reinterpret_cast<const float*>(u_W) + (size_t)(row0 >> 7) * f_pitch,
                           (uint32_t)f_pitch * 4u, &full[slot], pol);
         } else if (TMAP) {
           const int per_half = t_nrb * t_ncg;
@@ -988,7 +1004,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       const bool up = hd.kind == kKindUp;
       const bool sh = hd.seg == 0;
       const int Iu = sh ? args.Is : args.I;
-      const int lw = class_lw(hd.cls);
+      const int lw = geo_lw(hd.cls, FP8);
       const int c0 = hd.cp * (up ? lw / 2 : lw);
       const int w = min(up ? lw / 2 : lw, (up ? Iu : H) - c0);
       // local layout of the stage: UP gate [0, w), up [uoff, uoff + w); DOWN [0, w)
@@ -1002,9 +1018,10 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
           for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
       }
       const uint32_t sw = smem_addr(stages + (size_t)slot * kStageBytesMma);
-      const uint32_t sx = sw + kStageWBytes;
+      const uint32_t sx = sw + (FP8 ? fp8_stage_xoff(hd.cls) : kStageWBytes);
       if constexpr (FP8) {
-        const float* srow = reinterpret_cast<const float*>(stages + (size_t)slot * kStageBytesMma + kFp8StageWBytes);
+        const float* srow =
+            reinterpret_cast<const float*>(stages + (size_t)slot * kStageBytesMma + fp8_stage_wbytes(hd.cls));
         if (hd.cls == 0)
           mma_stage_fp8<0, NF, CW>(acc, sw, sx, srow, LW, hd.nrows, ntiles, up, c0, uoff, Iu, warp, lane);
         else if constexpr (KC >= 1) {
@@ -1040,12 +1057,12 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
         const size_t ld = up ? 2 * (size_t)Iu : (size_t)H;
         if (!warp_aborted(abort_flag)) {
           if (cls == 0)
-            flush_piece<0, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
+            flush_piece<0, NF, CW, FP8>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
           else if constexpr (KC >= 1) {
             if (cls == 1)
-              flush_piece<1, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
+              flush_piece<1, NF, CW, FP8>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
             else if constexpr (KC >= 2)
-              flush_piece<2, NF, CW>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
+              flush_piece<2, NF, CW, FP8>(acc, fbase, ld, my_row, my_wt, ntok, up, c0, w, uoff, LW, Iu, warp, lane);
           }
         }
         if (up) {

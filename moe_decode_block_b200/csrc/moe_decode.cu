@@ -233,18 +233,19 @@ bool encode_matrix_map(uint8_t* out, const void* base, int rows, int cols) {
 
 // Tensor map of an e4m3 matrix [rows, cols] stored row-major ([out, in]: a
 // row holds one output's weights over the inputs), seen as the 2-D tensor
-// {cols, rows} with {32, 256} boxes (32 bytes of inputs x 256 outputs) and
-// 32-byte swizzling (see mma_stage_fp8).
+// {cols, rows} with {128, 128} boxes (128 bytes of inputs x 128 outputs) and
+// 128-byte swizzling (see mma_stage_fp8).
 bool encode_fp8_map(uint8_t* out, const void* base, int rows, int cols) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc || cols % 16) return false;
   CUtensorMap m;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols};
-  cuuint32_t box[2] = {32, 256};
+  // one load: 128 input bytes (one line) of 128 output rows, 128-byte swizzle
+  cuuint32_t box[2] = {128, 128};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return false;
   std::memcpy(out, &m, sizeof m);

@@ -70,7 +70,10 @@ class Run:
 # 64 KB weight stage), restated to predict the device-side stage counters.
 CLASS_LW = (2048, 1024, 512)
 CLASS_ROWS = (16, 32, 64)
-CLASS_ROWS_FP8 = (32, 64, 64)  # stages of e4m3 weights
+# e4m3 weights: 128 input rows (one 128-byte line per weight row) by 512,
+# 512 and 256 columns
+CLASS_LW_FP8 = (512, 512, 256)
+ROWS_FP8 = 128
 UNIT_TOKENS = 32
 
 
@@ -81,7 +84,7 @@ def token_class(n):
 def unit_stages(c, up, H, I, fp8=False):
     """Stages of a unit's UP list (panels of lw/2 gate + up columns, r-row
     stages) or DOWN list (panels of lw columns, r-row stages)."""
-    lw, r = CLASS_LW[c], (CLASS_ROWS_FP8 if fp8 else CLASS_ROWS)[c]
+    lw, r = (CLASS_LW_FP8[c], ROWS_FP8) if fp8 else (CLASS_LW[c], CLASS_ROWS[c])
     cdiv = lambda a, b: -(-a // b)
     if up:
         return cdiv(I, lw // 2) * cdiv(H, r)
