@@ -24,23 +24,23 @@
 //   A: UP stages of the shared expert's units;
 //   B: UP stages of the routed units, DOWN stages of the shared units, DOWN
 //      stages of the routed units.
-// Segment A needs nothing from the router, so it runs *before* the
-// grid-dependency wait and overlaps the router kernel (launched just before
-// this one under programmatic dependent launch); a producer calls the wait
-// only when its ticket reaches segment B, whose length it then reads from the
-// plan.  CTAs pull chunks of stages from a global ticket counter.  Segment A
-// goes out in one round of a chunk per CTA; in segment B the first three
-// quarters go out in chunks of T/(4G) stages (at most 64),
-// the next 3/16 in quarter chunks, the rest one at a time, so the grid needs
-// no co-residency and ends with a tail of about one stage.  A DOWN stage
-// reads activation rows [row0, row0 + R), which one UP panel of its unit
-// produces; it is issued once that panel is published (a per-panel flag
-// holding the launch epoch, so flags never need clearing).  Every UP stage is
-// handed out before any DOWN stage, so the CTAs that still owe UP work are
-// running and the wait always ends (it is bounded all the same).  The shared
-// expert's DOWN stages would wait for its UP panels if they followed them in
-// segment A (a CTA that starts late, on the SM where the router's last CTA
-// ran, can hold the last of them); after the routed UP stages they are ready.
+// Segment A needs nothing from the router, so it runs while the router
+// kernel (launched just before this one under programmatic dependent launch)
+// computes the plan; a producer waits for the plan (its ready flag) only when
+// its ticket reaches segment B, whose length it then reads from the plan.
+// CTAs pull chunks of stages from a global ticket counter.  Segment A goes
+// out in one round of a chunk per CTA; in segment B the first three quarters
+// go out in chunks of T/(4G) stages (at most 64), the next 3/16 in quarter
+// chunks, the rest one at a time, so the grid needs no co-residency and ends
+// with a tail of about one stage.  A DOWN stage reads activation rows [row0,
+// row0 + R), which one UP panel of its unit produces; it is issued once that
+// panel is published (a per-panel flag holding the launch epoch, so flags
+// never need clearing).  Every UP stage is handed out before any DOWN stage,
+// so the CTAs that still owe UP work are running and the wait always ends (it
+// is bounded all the same).  The shared expert's DOWN stages stay after the
+// routed UP stages: placed right after its UP round (segment A), they waited
+// for the last UP chunks of each panel with nothing else to stream, which
+// measured slower at every batch size.
 // The producer keeps the plan (unit list, assignment slots) and the panels it
 // has seen published in shared memory: at every chunk change it would
 // otherwise walk the plan with chains of dependent L2 reads, and as all CTAs
@@ -196,6 +196,7 @@ struct MmaArgs {
   unsigned* panel_cnt_s;     // shared expert: [n_su * panel_stride_s]
   unsigned* panel_ready_s;
   unsigned* queue;           // [0] ticket counter, [1] finished CTAs (zero between calls), [2] launch epoch
+  int* plan_ready;           // the plan's ready flag (set by the router), returned to zero by the last CTA out
   int* status;
   uint32_t spin_limit;       // probes before a bounded wait gives up
   int hold_panel;            // testing only: routed UP panel whose publication is withheld (-1: none)
@@ -660,36 +661,47 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
     bool b_known = !args.has_routed;
     int n_units_r = 0;
     auto know_b = [&]() {
-      cudaGridDependencySynchronize();  // the plan is written by the router kernel
+      // The plan is written by the router kernel, whose last CTA sets its
+      // ready flag (release) once it is complete: poll that rather than wait
+      // for the router grid to complete.  Every router CTA is resident (this
+      // grid was launched once all of them had started), so the flag comes;
+      // the wait is bounded all the same.
       const Plan* pl = args.plan;
-      int n = __ldcg(&pl->n_active);
-      if (n < 0 || n > args.max_units) {
-        if (lane == 0) atomicCAS(args.status, kStatusOk, kStatusPlan);
-        n = 0;
-      }
-      n_units_r = n;
-      // copy the plan to shared memory, sanitised: an entry the router never
-      // produces is flagged and replaced by one that keeps every access in
-      // bounds
-      const int nas = B * args.top_k;
-      bool bad = false;
-      int T = 0;  // at most ~0.5M stages: 32-bit arithmetic
-      for (int u = lane; u < n; u += 32) {
-        int cnt = __ldcg(&pl->unit_count[u]);
-        int ex = __ldcg(&pl->unit_expert[u]);
-        int bg = __ldcg(&pl->unit_begin[u]);
-        if (cnt < 0 || cnt > kUnitTok || ex < 0 || ex >= args.E || bg < 0 || bg + cnt > nas) {
-          bad = true;
-          cnt = 0;
-          ex = 0;
-          bg = 0;
+      int ok = 1;
+      if (lane == 0) {
+        uint32_t it = 0;
+        while (ld_acquire_u32(reinterpret_cast<const unsigned*>(&pl->ready)) == 0u) {
+          if (++it > (uint32_t)s_misc[1] || *abort_flag) {
+            atomicCAS(args.status, kStatusOk, kStatusTimeout);
+            *abort_flag = 1;
+            ok = 0;
+            break;
+          }
+          __nanosleep(32);
         }
-        s_ucnt[u] = (uint8_t)cnt;
-        s_uexp[u] = (uint16_t)ex;
-        s_ubeg[u] = (uint16_t)bg;
-        const int c = cls_of(cnt);
-        T += unit_stages(c, true, H, args.I, FP8) + unit_stages(c, false, H, args.I, FP8);
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // copy the plan to shared memory in one round of loads: every unit
+      // entry the batch can produce and every assignment slot are loaded
+      // together with the unit count (entries past it are never used), then
+      // sanitised: an entry the router never produces is flagged and
+      // replaced by one that keeps every access in bounds
+      const int nas = B * args.top_k;
+      const int u_cap = min(args.max_units, nas);
+      int n = ok ? __ldcg(&pl->n_active) : 0;
+      // (stored so that a negative or oversized value stays out of range and
+      // is caught below: count 255 > kUnitTok, begin 0xffff > nas, a
+      // negative expert id >= 32768 > E)
+#pragma unroll 4
+      for (int u = lane; u < u_cap; u += 32) {
+        const int cnt = __ldcg(&pl->unit_count[u]), ex = __ldcg(&pl->unit_expert[u]),
+                  bg = __ldcg(&pl->unit_begin[u]);
+        s_ucnt[u] = (uint8_t)(cnt < 0 ? 255 : min(cnt, 255));
+        s_uexp[u] = (uint16_t)(ex < 0 ? 0xffff : min(ex, 0xffff));
+        s_ubeg[u] = (uint16_t)(bg < 0 ? 0xffff : min(bg, 0xffff));
+      }
+      bool bad = false;
+#pragma unroll 4
       for (int i = lane; i < nas; i += 32) {
         int sl = __ldcg(&pl->assign_slot[i]);
         if (sl < 0 || sl >= nas) {
@@ -697,6 +709,27 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
           sl = 0;
         }
         s_aslot[i] = (uint16_t)sl;
+      }
+      if (n < 0 || n > u_cap) {
+        if (lane == 0 && ok) atomicCAS(args.status, kStatusOk, kStatusPlan);
+        n = 0;
+      }
+      n_units_r = n;
+      __syncwarp();
+      int T = 0;  // at most ~0.5M stages: 32-bit arithmetic
+      for (int u = lane; u < n; u += 32) {
+        int cnt = s_ucnt[u], ex = s_uexp[u], bg = s_ubeg[u];
+        if (cnt > kUnitTok || ex >= args.E || bg + cnt > nas) {
+          bad = true;
+          cnt = 0;
+          ex = 0;
+          bg = 0;
+          s_ucnt[u] = 0;
+          s_uexp[u] = 0;
+          s_ubeg[u] = 0;
+        }
+        const int c = cls_of(cnt);
+        T += unit_stages(c, true, H, args.I, FP8) + unit_stages(c, false, H, args.I, FP8);
       }
       if (__any_sync(0xffffffffu, bad) && lane == 0) atomicCAS(args.status, kStatusOk, kStatusPlan);
 #pragma unroll
@@ -931,6 +964,9 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
       if (stop) break;
       tk = __shfl_sync(0xffffffffu, tk_next, 0);
     }
+    // the router grid ended long ago: wait for it formally, so nothing after
+    // this grid on the stream can overlap it
+    cudaGridDependencySynchronize();
     // tell the consumers there is no more work.  Only into a slot the
     // consumers have handed back: if that wait gave up, a stage may still
     // own the slot (its header in use, its barrier's phase not complete),
@@ -1139,6 +1175,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       args.queue[0] = 0u;
       args.queue[1] = 0u;
       args.queue[2] = args.queue[2] + 1u;
+      if (args.has_routed) *args.plan_ready = 0;
     }
   }
 }

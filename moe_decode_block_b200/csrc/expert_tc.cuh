@@ -427,6 +427,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       args.queue[0] = 0u;
       args.queue[1] = 0u;
       args.queue[2] = args.queue[2] + 1u;
+      if (args.has_routed) *args.plan_ready = 0;
     }
   }
 }

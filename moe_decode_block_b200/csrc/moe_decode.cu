@@ -501,6 +501,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.maps13_s = maps + 2 * (size_t)s.n_experts * mb;
   base.maps2_s = maps + (2 * (size_t)s.n_experts + 1) * mb;
   base.plan = h->at<Plan>(h->L.plan);
+  base.plan_ready = &h->at<Plan>(h->L.plan)->ready;
   base.x = static_cast<const __nv_bfloat16*>(x);
   base.h = h->at<float>(h->L.h);
   base.a = h->at<__nv_bfloat16>(h->L.a);

@@ -33,10 +33,13 @@ constexpr uint32_t kSpinLimit = 1u << 24;
 // Units follow the active experts in ascending id order (an expert with more
 // than kMaxUnitTokens tokens gets several consecutive units); the
 // assignments of unit u are [unit_begin[u], unit_begin[u] + unit_count[u]),
-// sorted by token.
+// sorted by token.  `ready` is set (release store) once the rest is written;
+// the expert kernel polls it instead of waiting for the router grid to
+// complete, and its last CTA returns it to zero.
 struct Plan {
   int n_active;  // number of units
-  int pad_[3];
+  int ready;
+  int pad_[2];
   int unit_expert[kMaxUnits];
   int unit_begin[kMaxUnits];
   int unit_count[kMaxUnits];

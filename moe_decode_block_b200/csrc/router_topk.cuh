@@ -486,7 +486,12 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
       __syncwarp();
     }
   }
+  // publish: every thread's plan writes, then the flag the expert kernel's
+  // producers poll (sooner than this grid's completion)
+  __threadfence();
+  __syncthreads();
   if (tid == 0) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(&a.plan->ready), "r"(1u) : "memory");
     *a.ticket = 0u;
     if (a.logits_stride > 0) *a.epoch = *a.epoch + 1u;  // every CTA read it before taking its ticket
   }
