@@ -141,9 +141,10 @@ typedef struct moe_decode_ctx* moe_decode_t;
  *                       expert)
  *   last_token_tiles  : token tiles of 8 the expert kernels were prepared for
  *                       in the last forward (ceil(min(batch, 32) / 8))
- * Device side (counted by the expert kernels as they run, cumulative since
- * moe_decode_init, graph replays included):
- *   stages_up[c], stages_down[c] : 64 KB weight stages the expert kernels
+ * Device side (added by the last CTA of each expert-kernel launch from the
+ * plan it consumed, cumulative since moe_decode_init, graph replays included):
+ *   stages_up[c], stages_down[c] : weight stages (64 KB; 32 KB for e4m3
+ *                       weights in class 2) the expert kernels
  *                       streamed for units of token class c (0: 1-8 tokens,
  *                       1: 9-16, 2: 17-32), up and down projections -- which
  *                       variants actually ran.

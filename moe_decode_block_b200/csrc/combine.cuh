@@ -14,48 +14,12 @@
 
 namespace moe {
 
-// What the combine kernel needs to count, per token class, the weight
-// stages the expert kernels streamed (from the plan they consumed).
-struct StageCountArgs {
-  const Plan* plan;                  // the routed units (nullptr: no routed pass)
-  unsigned long long* counts;        // [kNumClasses * 2]: UP, DOWN per class, cumulative
-  int n_su, batch, H, I, Is, kc, max_units, fp8;
-};
-
-// out[t, c] = bf16_rne(x[t, c] + acc[t, c]); acc returns to zero.  Warp 0 of
-// CTA 0 also adds the stages of this forward's units to the per-class
-// counters (device-side evidence of which token classes ran), off the
-// expert kernels' paths.
+// out[t, c] = bf16_rne(x[t, c] + acc[t, c]); acc returns to zero.
 __global__ void __launch_bounds__(256) combine_residual_kernel(const __nv_bfloat16* __restrict__ x,
                                                                float* __restrict__ acc,
-                                                               __nv_bfloat16* __restrict__ out, int n_vec8,
-                                                               const __grid_constant__ StageCountArgs sc) {
+                                                               __nv_bfloat16* __restrict__ out, int n_vec8) {
   cudaGridDependencySynchronize();
   cudaTriggerProgrammaticLaunchCompletion();
-  if (blockIdx.x == 0 && threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    unsigned long long c[2 * kNumClasses] = {};
-    auto add = [&](int n, int I) {
-      const int cls = min(class_for_tokens(n), sc.kc);
-      const unsigned long long u = (unsigned long long)unit_stages(cls, true, sc.H, I, sc.fp8 != 0);
-      const unsigned long long d = (unsigned long long)unit_stages(cls, false, sc.H, I, sc.fp8 != 0);
-#pragma unroll
-      for (int j = 0; j < kNumClasses; ++j) {
-        c[2 * j] += cls == j ? u : 0ull;
-        c[2 * j + 1] += cls == j ? d : 0ull;
-      }
-    };
-    for (int su = lane; su < sc.n_su; su += 32) add(min(kMaxUnitTokens, sc.batch - su * kMaxUnitTokens), sc.Is);
-    if (sc.plan) {
-      const int n = min(max(__ldcg(&sc.plan->n_active), 0), sc.max_units);
-      for (int u = lane; u < n; u += 32) add(min(max(__ldcg(&sc.plan->unit_count[u]), 0), kMaxUnitTokens), sc.I);
-    }
-#pragma unroll
-    for (int j = 0; j < 2 * kNumClasses; ++j) {
-      const unsigned long long v = __reduce_add_sync(0xffffffffu, (unsigned)c[j]);
-      if (lane == 0 && v) atomicAdd(&sc.counts[j], v);
-    }
-  }
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n_vec8) return;
   const uint4 xv = reinterpret_cast<const uint4*>(x)[i];

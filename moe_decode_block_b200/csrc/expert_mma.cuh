@@ -197,6 +197,7 @@ struct MmaArgs {
   unsigned* panel_ready_s;
   unsigned* queue;           // [0] ticket counter, [1] finished CTAs (zero between calls), [2] launch epoch
   int* plan_ready;           // the plan's ready flag (set by the router), returned to zero by the last CTA out
+  unsigned long long* stage_counts;  // [kNumClasses * 2]: UP, DOWN stages per token class, cumulative
   int* status;
   uint32_t spin_limit;       // probes before a bounded wait gives up
   int hold_panel;            // testing only: routed UP panel whose publication is withheld (-1: none)
@@ -613,6 +614,36 @@ __device__ __forceinline__ SmemView carve_smem(uint8_t* raw, int NS) {
   return v;
 }
 
+// The last CTA out adds the launch's stages per token class to the device
+// counters (evidence of which token classes ran): its copy of the plan is in
+// shared memory, as every producer reads the plan before it runs out of
+// tickets.  Warp 0, after the CTA's final barrier; one class at a time.
+template <int KC, bool FP8>
+__device__ __forceinline__ void count_stages_at_exit(const MmaArgs& args, const SmemView& sv, int lane) {
+  const int H = args.H, B = args.batch;
+  const int n_r = args.has_routed ? sv.s_misc[4] : 0;
+#pragma unroll 1
+  for (int j = 0; j < kNumClasses; ++j) {
+    unsigned up_st = 0, dn_st = 0;
+    for (int su = lane; su < args.n_su; su += 32) {
+      if (min(class_for_tokens(min(kUnitTok, B - su * kUnitTok)), KC) == j) {
+        up_st += unit_stages(j, true, H, args.Is, FP8);
+        dn_st += unit_stages(j, false, H, args.Is, FP8);
+      }
+    }
+    for (int u = lane; u < n_r; u += 32) {
+      if (min(class_for_tokens((int)sv.s_ucnt[u]), KC) == j) {
+        up_st += unit_stages(j, true, H, args.I, FP8);
+        dn_st += unit_stages(j, false, H, args.I, FP8);
+      }
+    }
+    up_st = __reduce_add_sync(0xffffffffu, up_st);
+    dn_st = __reduce_add_sync(0xffffffffu, dn_st);
+    if (lane == 0 && up_st) atomicAdd(&args.stage_counts[2 * j], (unsigned long long)up_st);
+    if (lane == 0 && dn_st) atomicAdd(&args.stage_counts[2 * j + 1], (unsigned long long)dn_st);
+  }
+}
+
 // The producer warp: takes tickets, walks the work list and fills the stage
 // ring (weights by TMA, the stage's token activations, the stage header);
 // ends by posting a kKindEnd header.  Shared by both expert kernels.
@@ -737,6 +768,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
       __syncwarp();
       sch_B = make_sched(T + S_dn, G, 4, args.stagger);
       b_known = true;
+      if (lane == 0) s_misc[4] = n;  // routed units, for the stage counters at exit
     };
     // Cursor over the work list: group (0 shared UP, 1 routed UP, 2 shared
     // DOWN, 3 routed DOWN), unit, and the list positions
@@ -1170,6 +1202,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
     // the last CTA out returns the counters to zero and advances the epoch
     __threadfence();
     const unsigned done = atomicAdd(&args.queue[1], 1u);
+    s_misc[5] = done == gridDim.x - 1 ? 1 : 0;
     if (done == gridDim.x - 1) {
       __threadfence();
       args.queue[0] = 0u;
@@ -1178,6 +1211,8 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
       if (args.has_routed) *args.plan_ready = 0;
     }
   }
+  __syncthreads();
+  if (warp == 0 && s_misc[5] && !*abort_flag) count_stages_at_exit<KC, FP8>(args, sv, lane);
 }
 
 }  // namespace moe

@@ -422,6 +422,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     __threadfence();
     const unsigned done = atomicAdd(&args.queue[1], 1u);
+    s_misc[5] = done == gridDim.x - 1 ? 1 : 0;
     if (done == gridDim.x - 1) {
       __threadfence();
       args.queue[0] = 0u;
@@ -430,6 +431,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (args.has_routed) *args.plan_ready = 0;
     }
   }
+  __syncthreads();
+  if (warp == 0 && s_misc[5] && !*abort_flag) count_stages_at_exit<2, false>(args, sv, lane);
 }
 
 }  // namespace moe

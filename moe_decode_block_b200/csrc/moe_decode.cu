@@ -502,6 +502,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   base.maps2_s = maps + (2 * (size_t)s.n_experts + 1) * mb;
   base.plan = h->at<Plan>(h->L.plan);
   base.plan_ready = &h->at<Plan>(h->L.plan)->ready;
+  base.stage_counts = h->at<unsigned long long>(h->L.stage_counts);
   base.x = static_cast<const __nv_bfloat16*>(x);
   base.h = h->at<float>(h->L.h);
   base.a = h->at<__nv_bfloat16>(h->L.a);
@@ -549,24 +550,10 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
     return mark(1, sm);
   };
 
-  // the combine kernel also counts the stages of this forward's units per
-  // token class (from the plan the expert kernels consumed)
-  moe::StageCountArgs sc{};
-  sc.plan = h->at<Plan>(h->L.plan);
-  sc.counts = h->at<unsigned long long>(h->L.stage_counts);
-  sc.n_su = n_su;
-  sc.batch = batch;
-  sc.H = s.hidden;
-  sc.I = s.inter;
-  sc.Is = s.n_shared ? s.shared_inter : 0;
-  sc.kc = h->use_tc ? moe::kNumClasses - 1 : kc;
-  sc.max_units = (int)max_units(&s);
-  sc.fp8 = f8 ? 1 : 0;
   auto launch_combine = [&](bool pdl) -> cudaError_t {
     const int nvec = batch * s.hidden / 8;
     cudaError_t err = launch(moe::combine_residual_kernel, ceil_div(nvec, 256), 256, 0, sm, pdl,
-                             static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec,
-                             sc);
+                             static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec);
     if (err != cudaSuccess) return err;
     ++kernels;
     return mark(3, sm);
