@@ -118,6 +118,21 @@ extern "C" {
  * An extension beyond the pages, which do not discuss weight precision.
  */
 #define MOE_FLAG_FP8_WEIGHTS 8u
+/*
+ * MOE_FLAG_PARTIAL_SUM: the forward writes, instead of bf16(x + sum), the
+ * fp32 sum of the expert outputs alone (routed, weighted, plus the shared
+ * expert; no residual, no rounding): `out` is then float32 [batch, hidden].
+ * For a tensor-parallel block: rank r's handle is made with inter /
+ * shared_inter divided by the TP size and given the rank's slices of every
+ * expert (w13: gate columns and up columns [r*I/tp, (r+1)*I/tp) each, w2:
+ * the same rows), so the ranks' partial sums add up to the block's expert
+ * sum; moe_decode_reduce_residual then forms bf16(x + sum over ranks).  The
+ * routing must agree across ranks (same x and router weights; the tests
+ * draw inputs whose top-k has a margin).  Not with moe_decode_forward_host.
+ * The pages run the block tensor-parallel across GPUs with the expert sum
+ * exchanged over NVLink ("Recovering time between operators").
+ */
+#define MOE_FLAG_PARTIAL_SUM 16u
 typedef struct moe_decode_shapes {
   int32_t hidden;
   int32_t n_experts;
@@ -253,6 +268,30 @@ int moe_decode_forward_fp8(moe_decode_t h, const void* x, const void* router_w, 
                            const void* shared_w13q, const void* shared_w13s, const void* shared_w2q,
                            const void* shared_w2s, void* out, int32_t* topk_ids, float* topk_w, int32_t batch,
                            void* stream_main, void* stream_aux);
+
+/*
+ * out[t, c] = bf16_rne(x[t, c] + sum_{r < n_parts} partials[r][t, c]), the
+ * residual step of a tensor-parallel block with the all-reduce of the ranks'
+ * partial sums folded in: partials[r] are the fp32 [batch, hidden] outputs
+ * of MOE_FLAG_PARTIAL_SUM forwards -- device pointers, which on an
+ * NVLink/NVSwitch system may be peer memory (another GPU's buffer mapped
+ * into this device's address space), so every rank reads all ranks' sums
+ * directly.  The sum is taken in the order r = 0 .. n_parts-1, so every
+ * rank computes the same bits.  The caller orders the partials' producers
+ * before this launch (stream order, or an event / barrier across devices).
+ *   partials : HOST array of n_parts device pointers, 16-byte aligned
+ *   n_parts  : 1 .. MOE_REDUCE_MAX_PARTS
+ *   x, out   : device, bf16 [batch, hidden], 16-byte aligned (out may alias x)
+ *   batch, hidden : 1 .. 64, multiple of 8 up to 16384
+ *   stream   : cudaStream_t, NULL = legacy default stream
+ * Asynchronous.  Errors: MOE_ERR_INVALID_ARG (NULL or misaligned pointer,
+ * n_parts or sizes out of range), MOE_ERR_NO_DEVICE, MOE_ERR_CUDA.
+ * No counterpart in the pages' API; it is this library's form of the
+ * NVLink exchange the pages describe.
+ */
+#define MOE_REDUCE_MAX_PARTS 16
+int moe_decode_reduce_residual(const void* const* partials, int32_t n_parts, const void* x, void* out,
+                               int32_t batch, int32_t hidden, void* stream);
 
 /* Free the workspace and events; NULL is accepted.  Waits for the handle's
  * work first, as moe_decode_get_status does. */

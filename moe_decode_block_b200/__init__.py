@@ -35,13 +35,15 @@ EXPORTED = (
     "moe_decode_get_status", "moe_decode_get_stats", "moe_decode_error_string",
     "moe_decode_last_cuda_error", "moe_decode_last_cuda_error_string", "moe_decode_workspace_bytes",
     "moe_decode_set_timing_events", "moe_decode_set_wait_limit", "moe_router_topk_noalloc",
-    "moe_router_topk_noalloc_status",
+    "moe_router_topk_noalloc_status", "moe_decode_reduce_residual",
 )
 MOE_TIMING_EVENTS = 6
 MOE_FLAG_TWO_STREAM = 1
 MOE_FLAG_TCGEN05 = 2
 MOE_FLAG_TEST_HOLD_PANEL = 4
 MOE_FLAG_FP8_WEIGHTS = 8
+MOE_FLAG_PARTIAL_SUM = 16
+MOE_REDUCE_MAX_PARTS = 16
 
 
 class Shapes(ctypes.Structure):
@@ -112,6 +114,8 @@ def load_library() -> ctypes.CDLL:
     lib.moe_router_topk_noalloc.restype = I
     lib.moe_router_topk_noalloc_status.argtypes = [P]
     lib.moe_router_topk_noalloc_status.restype = I
+    lib.moe_decode_reduce_residual.argtypes = [P, ctypes.c_int32, P, P, ctypes.c_int32, ctypes.c_int32, P]
+    lib.moe_decode_reduce_residual.restype = I
     lib.moe_decode_set_wait_limit.argtypes = [P, ctypes.c_uint32]
     lib.moe_decode_set_wait_limit.restype = I
     lib.moe_decode_workspace_bytes.argtypes = [ctypes.POINTER(Shapes)]
@@ -165,23 +169,40 @@ def router_topk_noalloc_status(stream=None) -> int:
     return lib.moe_router_topk_noalloc_status(sm)
 
 
+def reduce_residual(partials, x, out, stream=None):
+    """out = bf16(x + sum of the fp32 [B, H] partial sums in `partials`, in
+    list order) -- moe_decode_reduce_residual; the tensors (or raw device
+    pointers, e.g. a peer's mapped buffer) must be 16-byte aligned."""
+    import torch
+    lib = load_library()
+    ptrs = (ctypes.c_void_p * len(partials))(*[_ptr(p) if hasattr(p, "data_ptr") else int(p) for p in partials])
+    sm = _stream_handle(stream if stream is not None else torch.cuda.current_stream())
+    rc = lib.moe_decode_reduce_residual(ptrs, len(partials), _ptr(x), _ptr(out), int(x.shape[0]), int(x.shape[1]),
+                                        sm)
+    _check(rc, "moe_decode_reduce_residual")
+
+
 class MoEDecode:
     """One MoE block shape bound to the current CUDA device (owns a workspace).
 
     two_stream=False (default): router kernel, one expert kernel (shared
     and routed experts) and the combine on the main stream.  two_stream=True:
     MOE_FLAG_TWO_STREAM, the shared expert on the aux stream.  tcgen05=True:
-    MOE_FLAG_TCGEN05, the expert kernel on tcgen05 with TMEM accumulators."""
+    MOE_FLAG_TCGEN05, the expert kernel on tcgen05 with TMEM accumulators.
+    fp8=True: MOE_FLAG_FP8_WEIGHTS (forward_fp8).  partial=True:
+    MOE_FLAG_PARTIAL_SUM, `out` receives the fp32 expert sum without the
+    residual (one tensor-parallel rank's share; see tp.py)."""
 
     def __init__(self, hidden: int, n_experts: int, top_k: int, inter: int, shared_inter: int = 0,
                  n_shared: int = 1, max_batch: int = 64, router_bias=None, two_stream: bool = False,
-                 tcgen05: bool = False, extra_flags: int = 0, fp8: bool = False):
+                 tcgen05: bool = False, extra_flags: int = 0, fp8: bool = False, partial: bool = False):
         self._lib = load_library()
         self._bias = router_bias  # keep the device tensor alive
         self.two_stream = bool(two_stream)
         self.tcgen05 = bool(tcgen05)
         flags = (MOE_FLAG_TWO_STREAM if two_stream else 0) | (MOE_FLAG_TCGEN05 if tcgen05 else 0) | int(extra_flags)
         flags |= MOE_FLAG_FP8_WEIGHTS if fp8 else 0
+        flags |= MOE_FLAG_PARTIAL_SUM if partial else 0
         self.shapes = Shapes(hidden, n_experts, top_k, inter, shared_inter if n_shared else 0, n_shared,
                              max_batch, _ptr(router_bias), flags)
         h = ctypes.c_void_p()

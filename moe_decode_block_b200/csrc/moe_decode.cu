@@ -75,7 +75,8 @@ bool shapes_valid(const moe_decode_shapes* s) {
   if (s->n_shared != 0 && s->n_shared != 1) return false;
   if (s->n_shared == 1 && (!in(s->shared_inter, 8, 16384) || s->shared_inter % 8)) return false;
   if (!in(s->max_batch, 1, moe::kMaxBatch)) return false;
-  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05 | MOE_FLAG_TEST_HOLD_PANEL | MOE_FLAG_FP8_WEIGHTS)) != 0)
+  if ((s->flags & ~(MOE_FLAG_TWO_STREAM | MOE_FLAG_TCGEN05 | MOE_FLAG_TEST_HOLD_PANEL | MOE_FLAG_FP8_WEIGHTS |
+                    MOE_FLAG_PARTIAL_SUM)) != 0)
     return false;
   if (s->flags & MOE_FLAG_FP8_WEIGHTS) {
     // e4m3 weights: whole 128 x 128 scale blocks, on the mma.sync kernel
@@ -551,9 +552,16 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   };
 
   auto launch_combine = [&](bool pdl) -> cudaError_t {
-    const int nvec = batch * s.hidden / 8;
-    cudaError_t err = launch(moe::combine_residual_kernel, ceil_div(nvec, 256), 256, 0, sm, pdl,
-                             static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec);
+    cudaError_t err;
+    if (s.flags & MOE_FLAG_PARTIAL_SUM) {  // the fp32 expert sum alone
+      const int nvec4 = batch * s.hidden / 4;
+      err = launch(moe::partial_sum_kernel, ceil_div(nvec4, 256), 256, 0, sm, pdl, base.acc, static_cast<float*>(out),
+                   nvec4);
+    } else {
+      const int nvec = batch * s.hidden / 8;
+      err = launch(moe::combine_residual_kernel, ceil_div(nvec, 256), 256, 0, sm, pdl,
+                   static_cast<const __nv_bfloat16*>(x), base.acc, static_cast<__nv_bfloat16*>(out), nvec);
+    }
     if (err != cudaSuccess) return err;
     ++kernels;
     return mark(3, sm);
@@ -1070,6 +1078,7 @@ int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* rout
                             void* out_host, int32_t* ids_host, float* w_host, int32_t batch, void* stream_main,
                             void* stream_aux) {
   if (h && (h->s.flags & MOE_FLAG_FP8_WEIGHTS)) return MOE_ERR_INVALID_ARG;  // bf16 weights only
+  if (h && (h->s.flags & MOE_FLAG_PARTIAL_SUM)) return MOE_ERR_INVALID_ARG;  // bf16 out only
   int rc = check_forward_args(h, x_host, router_w, w13, w2, shared_w13, shared_w2, out_host, ids_host, w_host,
                               batch, false);
   if (rc != MOE_OK) return rc;
@@ -1112,6 +1121,30 @@ int moe_decode_forward_host(moe_decode_t h, const void* x_host, const void* rout
   }
   if ((e = cudaStreamSynchronize(sm)) != cudaSuccess) return fail_cuda(e);
   return MOE_OK;
+}
+
+int moe_decode_reduce_residual(const void* const* partials, int32_t n_parts, const void* x, void* out,
+                               int32_t batch, int32_t hidden, void* stream) {
+  static_assert(MOE_REDUCE_MAX_PARTS == moe::kMaxReduceParts, "partials per reduction");
+  if (!partials || !x || !out) return MOE_ERR_INVALID_ARG;
+  if (n_parts < 1 || n_parts > MOE_REDUCE_MAX_PARTS) return MOE_ERR_INVALID_ARG;
+  if (batch < 1 || batch > moe::kMaxBatch || hidden < 8 || hidden > 16384 || hidden % 8) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  moe::PartialPtrs pp{};
+  for (int r = 0; r < n_parts; ++r) {
+    if (!partials[r] || !aligned16(partials[r])) return MOE_ERR_INVALID_ARG;
+    pp.p[r] = static_cast<const float*>(partials[r]);
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  const int nvec = batch * hidden / 8;
+  const cudaError_t e =
+      launch(moe::reduce_residual_kernel, ceil_div(nvec, 256), 256, 0, static_cast<cudaStream_t>(stream), false, pp,
+             (int)n_parts, static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(out), nvec);
+  return e == cudaSuccess ? MOE_OK : fail_cuda(e);
 }
 
 int moe_decode_destroy(moe_decode_t h) {

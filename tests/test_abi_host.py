@@ -65,7 +65,7 @@ def test_workspace_bytes_and_shape_validation(lib):
     assert 0 < tiny < full
     bad = [dict(hidden=7170), dict(hidden=0), dict(n_experts=12), dict(n_experts=2048), dict(top_k=0),
            dict(top_k=33), dict(top_k=9, n_experts=8), dict(inter=100), dict(n_shared=2),
-           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=16), dict(flags=17), dict(flags=1 << 31),
+           dict(shared_inter=12), dict(max_batch=0), dict(max_batch=65), dict(flags=32), dict(flags=33), dict(flags=1 << 31),
            dict(flags=8, hidden=7168 + 64), dict(flags=8, inter=2048 + 64), dict(flags=8 | 2)]
     for kw in bad:
         sh = _shapes(**kw)
@@ -82,6 +82,8 @@ def test_workspace_bytes_and_shape_validation(lib):
     # the testing-only hold flag is accepted too (the handle's first forward
     # withholds one panel publication)
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_TEST_HOLD_PANEL))) == full
+    # partial sums (one tensor-parallel rank's share) need no other workspace
+    assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(flags=mdb.MOE_FLAG_PARTIAL_SUM))) == full
     # shared_inter is ignored when there is no shared expert
     assert lib.moe_decode_workspace_bytes(ctypes.byref(_shapes(n_shared=0, shared_inter=0))) > 0
 
@@ -97,6 +99,19 @@ def test_null_arguments_are_rejected_on_the_host(lib):
     assert lib.moe_decode_forward_host(None, *([None] * 9), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_set_wait_limit(None, 100) == mdb.MOE_ERR_INVALID_ARG
     assert lib.moe_decode_forward_fp8(None, *([None] * 13), 1, None, None) == mdb.MOE_ERR_INVALID_ARG
+    # the reduce + residual step checks its arguments before touching a device
+    buf = ctypes.create_string_buffer(64 + 16)
+    a16 = (ctypes.addressof(buf) + 15) // 16 * 16
+    one = (ctypes.c_void_p * 1)(a16)
+    assert lib.moe_decode_reduce_residual(None, 1, a16, a16, 1, 8, None) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_reduce_residual(one, 0, a16, a16, 1, 8, None) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_reduce_residual(one, mdb.MOE_REDUCE_MAX_PARTS + 1, a16, a16, 1, 8,
+                                          None) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_reduce_residual(one, 1, a16 + 4, a16, 1, 8, None) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_reduce_residual(one, 1, a16, a16, 1, 12, None) == mdb.MOE_ERR_INVALID_ARG
+    assert lib.moe_decode_reduce_residual(one, 1, a16, a16, 65, 8, None) == mdb.MOE_ERR_INVALID_ARG
+    bad = (ctypes.c_void_p * 1)(a16 + 8)
+    assert lib.moe_decode_reduce_residual(bad, 1, a16, a16, 1, 8, None) == mdb.MOE_ERR_INVALID_ARG
 
 
 def test_init_without_a_gpu_reports_no_device(lib):
