@@ -69,6 +69,9 @@ def parse_args():
     p.add_argument("--no-configs", action="store_true", help="skip the other graded configurations")
     p.add_argument("--config-steps", type=int, default=200, help="timed graph replays per extra configuration")
     p.add_argument("--no-parity", action="store_true", help="skip the oracle check of the timed forwards")
+    p.add_argument("--fp8-forwards", type=int, default=0,
+                   help="profiling driver: run this many e4m3-weight forwards of the config (L2 flushed before "
+                        "each), print their event-timed us and exit (no bench line)")
     return p.parse_args()
 
 
@@ -445,6 +448,9 @@ def run_ours(args):
     wl = synth.WORKLOADS[args.config]
     s = wl.shape
     B = wl.batch
+    if args.fp8_forwards > 0:
+        fp8_forwards(wl, args.fp8_forwards, args.seed, dev)
+        return
     wts, x, margin = make_inputs(wl, args.seed, args.seed + 1000 * rank, dev)
     main = torch.cuda.Stream()
     aux = torch.cuda.Stream()
@@ -733,6 +739,38 @@ def run_ours(args):
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
     return 0 if parity_ok and status == 0 else 1
+
+
+def fp8_forwards(wl, n, seed, dev):
+    """Profiling driver for the e4m3-weight kernel: n forwards of the config's
+    block with e4m3 expert weights, L2 flushed before each (for ncu captures
+    of a small case; prints the event-timed us of each forward)."""
+    import torch
+    from moe_decode_block_b200 import MoEDecode, synth
+    s = wl.shape
+    w8 = synth.make_fp8_weights(s, seed=seed, device=dev, routing=wl.routing)
+    x = synth.make_x(wl.batch, s.hidden, seed=seed).to(dev)
+    blk = MoEDecode(s.hidden, s.n_experts, s.top_k, s.inter, s.shared_inter, n_shared=s.n_shared,
+                    max_batch=wl.batch, router_bias=w8.router_bias, fp8=True)
+    out = torch.empty_like(x)
+    ids = torch.empty(wl.batch, s.top_k, dtype=torch.int32, device=dev)
+    w = torch.empty(wl.batch, s.top_k, dtype=torch.float32, device=dev)
+    fb = torch.empty(2 * torch.cuda.get_device_properties(dev).L2_cache_size // 4, dtype=torch.float32, device=dev)
+    us = []
+    for _ in range(n):
+        fb.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        blk.forward_fp8(x, w8.router_w, w8.q13, w8.s13, w8.q2, w8.s2, w8.shared_q13, w8.shared_s13, w8.shared_q2,
+                        w8.shared_s2, out, ids, w)
+        e1.record()
+        torch.cuda.synchronize()
+        us.append(round(e0.elapsed_time(e1) * 1e3, 1))
+    status = blk.status()
+    blk.close()
+    print(json.dumps({"fp8_forwards": wl.name, "us": us, "device_status": status}), flush=True)
+    if status != 0:
+        raise SystemExit(f"device status {status}")
 
 
 def main():
