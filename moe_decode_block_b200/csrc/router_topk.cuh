@@ -317,6 +317,29 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
   for (int e = tid; e < E; e += NT) s_bias[e] = a.bias ? a.bias[e] : 0.f;
   const int nv = (E + 31) / 32;
   const int TB = router_stage_tokens(B, E);
+  constexpr int NWARP = NT / 32;
+  // one token whose logits all fit one per thread: the threshold top-k below
+  const bool one_token = B == 1 && E <= NT && k <= 8 && nv >= k;
+  // lanes j < k of a warp hold token t's selection in order: the ids, their
+  // renormalised weights p_j / sum_S p = exp(l_j - l_max) / sum_S exp(l_i - l_max)
+  auto finish_token = [&](int t, int my_id, float my_v) {
+    if (lane < k && (my_id < 0 || my_id >= E)) {  // cannot happen for k <= E; keep the plan valid
+      atomicCAS(a.status, kStatusOk, kStatusPlan);
+      my_id = lane;
+    }
+    const float lmax = __shfl_sync(0xffffffffu, my_v, 0);
+    const float ex = (lane < k) ? expf(my_v - lmax) : 0.f;
+    float sum = ex;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane < k) {
+      const float wj = ex / sum;
+      a.topk_ids[(size_t)t * k + lane] = my_id;
+      a.topk_w[(size_t)t * k + lane] = wj;
+      s_ids[t * k + lane] = my_id;
+      s_w[t * k + lane] = wj;
+    }
+  };
   for (int tb0 = 0; tb0 < B; tb0 += TB) {
     const int ntb = min(TB, B - tb0);
     {
@@ -342,6 +365,90 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
       }
     }
     __syncthreads();
+  if (one_token) {
+    // One token, one logit per thread.  The k-th largest of the warps' maxima
+    // is a threshold no member of the top k lies below (k real values reach
+    // it); the values at or above it -- a handful -- are collected and one
+    // warp sorts them by (value desc, id asc).  A few dependent steps across
+    // the whole CTA instead of one warp's long merge chain on the path the
+    // expert kernel waits for.  More than 32 candidates (ties on a large
+    // scale): the one-warp merge below.
+    float* w_max = s_w + kMaxAssign - 64;  // [NWARP + 1]: the warps' maxima, then the threshold
+    int* n_cand = s_ids + kMaxAssign - 64;
+    float* cand_v = s_w + kMaxAssign / 2;  // [32]
+    int* cand_i = s_ids + kMaxAssign / 2;
+    const float v = tid < E ? s_lg[tid] + s_bias[tid] : -INFINITY;
+    float m = v;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) w_max[warp] = m;
+    if (tid == 0) *n_cand = 0;
+    __syncthreads();
+    if (warp == 0) {
+      float mv = lane < NWARP ? w_max[lane] : -INFINITY;
+      // bitonic sort, descending
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, mv, stride);
+          const bool keep_max = ((lane & stride) == 0) == ((lane & size) == 0);
+          mv = keep_max ? fmaxf(mv, ov) : fminf(mv, ov);
+        }
+      }
+      if (lane == k - 1) w_max[NWARP] = mv;
+    }
+    __syncthreads();
+    const float thr = w_max[NWARP];
+    if (tid < E && v >= thr) {
+      const int p = atomicAdd(n_cand, 1);
+      if (p < 32) {
+        cand_v[p] = v;
+        cand_i[p] = tid;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const int nc = *n_cand;
+      int my_id = -1;
+      float my_v = -INFINITY;
+      if (nc <= 32) {
+        float cv = lane < nc ? cand_v[lane] : -INFINITY;
+        int ci = lane < nc ? cand_i[lane] : 0x7fffffff;
+        // bitonic sort, best first: larger value, then the smaller id
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+          for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, cv, stride);
+            const int oi = __shfl_xor_sync(0xffffffffu, ci, stride);
+            const bool other_better = ranks_before(ov, oi, cv, ci);
+            const bool keep_better = ((lane & stride) == 0) == ((lane & size) == 0);
+            if (keep_better == other_better) {
+              cv = ov;
+              ci = oi;
+            }
+          }
+        }
+        if (lane < k) {
+          my_id = ci;
+          my_v = cv;
+        }
+      } else {
+        float tv[8];
+        int ti[8];
+        warp_top8(s_lg, s_bias, E, lane, tv, ti);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          if (r == lane && r < k) {
+            my_id = ti[r];
+            my_v = tv[r];
+          }
+        }
+      }
+      finish_token(tb0, my_id, my_v);
+    }
+  } else
   for (int t = tb0 + warp; t < tb0 + ntb; t += NT / 32) {
     const float* lg = s_lg + (size_t)(t - tb0) * E;
     float v[NV];
@@ -383,10 +490,6 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
           my_v = tv[r];
         }
       }
-      if (lane < k && (my_id < 0 || my_id >= E)) {  // cannot happen for k <= E; keep the plan valid
-        atomicCAS(a.status, kStatusOk, kStatusPlan);
-        my_id = lane;
-      }
     } else {
     float lbv;
     int lbi;
@@ -409,19 +512,7 @@ __global__ void __launch_bounds__(router_threads(NV), 1) router_topk_kernel(cons
       }
     }
     }
-    // renormalised weights: p_j / sum_S p = exp(l_j - l_max) / sum_S exp(l_i - l_max)
-    const float lmax = __shfl_sync(0xffffffffu, my_v, 0);
-    const float ex = (lane < k) ? expf(my_v - lmax) : 0.f;
-    float sum = ex;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (lane < k) {
-      const float wj = ex / sum;
-      a.topk_ids[(size_t)t * k + lane] = my_id;
-      a.topk_w[(size_t)t * k + lane] = wj;
-      s_ids[t * k + lane] = my_id;
-      s_w[t * k + lane] = wj;
-    }
+    finish_token(t, my_id, my_v);
   }
     __syncthreads();  // the staging buffer is reused by the next group of tokens
   }
