@@ -475,9 +475,16 @@ __device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, 
     b[2] = h1 ? bf16x2_to_f16x2(v2) : 0u;
     b[3] = h1 ? bf16x2_to_f16x2(v3) : 0u;
   };
-  // one token tile: its fragments stay in registers for all m-tiles; more
-  // tiles: reloaded per m-tile (keeping them all costs spills)
+  // one token tile: its fragments stay in registers for all m-tiles, and the
+  // stage's products are summed over its 128 rows before the one scale
+  // multiply (a stage lies in one 128 x 128 block); more tiles: reloaded per
+  // m-tile (keeping them all costs spills) and scaled per product
   constexpr bool kKeepB = NT == 1;
+  float ts[kKeepB ? MT : 1][4];
+#pragma unroll
+  for (int mt = 0; mt < (kKeepB ? MT : 1); ++mt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ts[mt][j] = 0.f;
   // (the slice loop stays rolled: unrolled, its hoisted addresses and
   // fragments spill in the classes with several token tiles)
 #pragma unroll 1
@@ -493,13 +500,10 @@ __device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, 
         uint32_t r0, r1, r2, r3;
         ldsm_x4(sw + (uint32_t)(col * 128 + unit * 16), r0, r1, r2, r3);
         if (kKeepB) {
-          float t[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_f16_16816(t, e4m3x2_lo_to_f16x2(r0), e4m3x2_lo_to_f16x2(r1), e4m3x2_hi_to_f16x2(r0),
-                        e4m3x2_hi_to_f16x2(r1), bk[0], bk[1]);
-          mma_f16_16816(t, e4m3x2_lo_to_f16x2(r2), e4m3x2_lo_to_f16x2(r3), e4m3x2_hi_to_f16x2(r2),
-                        e4m3x2_hi_to_f16x2(r3), bk[2], bk[3]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[mt * NT][j] = fmaf(sc, t[j], acc[mt * NT][j]);
+          mma_f16_16816(ts[kKeepB ? mt : 0], e4m3x2_lo_to_f16x2(r0), e4m3x2_lo_to_f16x2(r1),
+                        e4m3x2_hi_to_f16x2(r0), e4m3x2_hi_to_f16x2(r1), bk[0], bk[1]);
+          mma_f16_16816(ts[kKeepB ? mt : 0], e4m3x2_lo_to_f16x2(r2), e4m3x2_lo_to_f16x2(r3),
+                        e4m3x2_hi_to_f16x2(r2), e4m3x2_hi_to_f16x2(r3), bk[2], bk[3]);
         } else {
           // half by half: one half's A fragment and one tile's B pair live
 #pragma unroll
@@ -524,6 +528,13 @@ __device__ __forceinline__ void mma_stage_fp8(float (&acc)[NF][4], uint32_t sw, 
         }
       }
     }
+  }
+  if (kKeepB) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+      if (m0 + mt * 16 < LW)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[mt * NT][j] = fmaf(sc, ts[kKeepB ? mt : 0][j], acc[mt * NT][j]);
   }
 }
 
