@@ -50,11 +50,18 @@
 // Panels.  Each matrix is cut into column panels and K-row stages of 64 KB
 // of weights.  A unit with n tokens takes the panel of its token class, the
 // narrower the more token tiles it has, so that a consumer warp's columns x
-// token tiles -- its accumulators -- stay the same in every class:
-//   class 0: n <=  8 : 2048 local columns, 16-row stages (1 token tile)
+// token tiles -- its accumulators -- stay within 32 fp32 registers:
+//   class 0: n <=  8 : 1024 local columns, 32-row stages (1 token tile)
 //   class 1: n <= 16 : 1024 local columns, 32-row stages (2 token tiles)
 //   class 2: n <= 32 :  512 local columns, 64-row stages (4 token tiles)
-// -- 16 consumer warps, each with 32 fp32 accumulators, in every instance.
+// -- 16 consumer warps in every instance, each with 16 (class 0 only) or 32
+// accumulators.  Class 0 is not the wider 2048 x 16 shape its one token tile
+// would allow: a hidden size of 7 x 1024 (7168) cuts into 2048-column DOWN
+// panels with a half-empty last one, and a stage costs about the same ring
+// time whatever its bytes (measured: the last panel's 32 KB stages landed
+// 0.9x as far apart as the full ones), so 1024 columns stream the DOWN list
+// in 7/8 of the stages; a piece (the split-K unit of work) also covers twice
+// the rows, which halves the partial sums flushed per weight byte.
 // A launch is compiled for the largest class its batch can produce (KC), so
 // small batches carry no code for the wider classes.  UP panels pair gate
 // columns [c0, c0 + LW/2) with up columns [I + c0, ...), so a panel holds
@@ -87,13 +94,12 @@ namespace moe {
 
 constexpr int kUnitTok = kMaxUnitTokens;  // tokens of one unit, at most
 constexpr int kNumClasses = 3;
-// Token classes.  A unit with more tokens takes a narrower panel of more
-// rows, so every stage holds lw x rows = 32K weights (64 KB) and every
-// consumer warp keeps the same eight accumulator fragments (32 floats) in
-// every class: 2048 x 16 for 1-8 tokens (one 8-token tile), 1024 x 32 for
-// 9-16 (two tiles), 512 x 64 for 17-32 (four tiles).
-__host__ __device__ constexpr int class_lw(int c) { return c == 0 ? 2048 : (c == 1 ? 1024 : 512); }
-__host__ __device__ constexpr int class_rows(int c) { return c == 0 ? 16 : (c == 1 ? 32 : 64); }
+// Token classes.  Every stage holds lw x rows = 32K weights (64 KB): 1024 x
+// 32 for 1-8 tokens (one 8-token tile) and for 9-16 (two tiles), 512 x 64
+// for 17-32 (four tiles); a consumer warp keeps four accumulator fragments
+// (16 floats) in class 0 and eight (32 floats) in classes 1 and 2.
+__host__ __device__ constexpr int class_lw(int c) { return c == 2 ? 512 : 1024; }
+__host__ __device__ constexpr int class_rows(int c) { return c == 2 ? 64 : 32; }
 __host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : 4); }
 // class of a unit with n <= kUnitTok tokens
 __host__ __device__ constexpr int class_for_tokens(int n) { return n <= 8 ? 0 : (n <= 16 ? 1 : 2); }
@@ -113,6 +119,7 @@ __host__ __device__ constexpr int geo_lw(int c, bool fp8) { return fp8 ? class_l
 __host__ __device__ constexpr int fp8_stage_wbytes(int c) { return class_lw_fp8(c) * kFp8Rows; }
 __host__ __device__ constexpr int fp8_stage_xoff(int c) { return fp8_stage_wbytes(c) + 1024; }
 constexpr int kFp8XPitch = kFp8Rows * 2 + 16;  // bytes per token row of activations
+__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 // Consumer warps: sixteen in every instance (seventeen warps with the
 // producer cap a thread at 96 registers, room for the 32 accumulators).
 __host__ __device__ constexpr int consumer_warps_for(int) { return 16; }
@@ -121,13 +128,15 @@ __host__ __device__ constexpr int expert_threads(int kc) { return (consumer_warp
 __host__ __device__ constexpr int class_mt(int c, int cw) { return class_lw(c) / (cw * 16); }
 __host__ __device__ constexpr int geo_mt(int c, int cw, bool fp8) { return geo_lw(c, fp8) / (cw * 16); }
 // accumulator fragments (of 4 floats) a consumer thread needs for classes <= KC
-__host__ __device__ constexpr int acc_frags(int kc) { return class_mt(0, consumer_warps_for(kc)) * class_nt(0); }
-static_assert(class_mt(1, 16) * class_nt(1) == acc_frags(1) && class_mt(2, 16) * class_nt(2) == acc_frags(2),
-              "every class keeps the same accumulators");
+__host__ __device__ constexpr int class_frags(int c, int cw) { return class_mt(c, cw) * class_nt(c); }
+__host__ __device__ constexpr int acc_frags(int kc) {
+  return kc <= 0 ? class_frags(0, consumer_warps_for(kc))
+                 : cmax(acc_frags(kc - 1), class_frags(kc, consumer_warps_for(kc)));
+}
+static_assert(acc_frags(0) == 4 && acc_frags(1) == 8 && acc_frags(2) == 8, "16 or 32 accumulators a thread");
 // stage buffers: weights (row pitch 2*lw + 16 on the plain-copy path) and
 // the tokens' activation rows (pitch 2*rows + 16), largest over the classes
 __host__ __device__ constexpr int stage_w_bytes(int c) { return class_rows(c) * (class_lw(c) * 2 + 16); }
-__host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 constexpr int kStageWBytes = cmax(stage_w_bytes(0), cmax(stage_w_bytes(1), stage_w_bytes(2)));  // 66560
 constexpr int kStageXBytes = kUnitTok * (class_rows(2) * 2 + 16);                                 // 4608
 constexpr int kStageBytesMma = (kStageWBytes + kStageXBytes + 1023) / 1024 * 1024;               // 70 KB
@@ -136,10 +145,9 @@ static_assert(fp8_stage_xoff(0) + 8 * kFp8XPitch <= kStageBytesMma &&
                   fp8_stage_xoff(1) + 16 * kFp8XPitch <= kStageBytesMma &&
                   fp8_stage_xoff(2) + 32 * kFp8XPitch <= kStageBytesMma,
               "fp8 stages: weights, scale row and the class's token rows fit one stage");
-static_assert(geo_mt(0, 16, true) * class_nt(0) <= class_mt(0, 16) * class_nt(0) &&
-                  geo_mt(1, 16, true) * class_nt(1) <= class_mt(0, 16) * class_nt(0) &&
-                  geo_mt(2, 16, true) * class_nt(2) <= class_mt(0, 16) * class_nt(0),
-              "fp8 classes need no more accumulators than the bf16 ones");
+static_assert(geo_mt(0, 16, true) * class_nt(0) <= acc_frags(0) && geo_mt(1, 16, true) * class_nt(1) <= acc_frags(1) &&
+                  geo_mt(2, 16, true) * class_nt(2) <= acc_frags(2),
+              "fp8 classes need no more accumulators than the bf16 instance of the same class");
 constexpr int kMaxStagesMma = 3;
 constexpr int kMaxChunk = 64;  // stages per queue grab, at most
 // tensor-map path: boxes of {64 columns, 16 rows, 4 column chunks}

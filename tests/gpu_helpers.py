@@ -68,8 +68,8 @@ class Run:
 
 # Panel geometry of the expert kernels' token classes (columns x rows of a
 # 64 KB weight stage), restated to predict the device-side stage counters.
-CLASS_LW = (2048, 1024, 512)
-CLASS_ROWS = (16, 32, 64)
+CLASS_LW = (1024, 1024, 512)
+CLASS_ROWS = (32, 32, 64)
 # e4m3 weights: 128 input rows (one 128-byte line per weight row) by 512,
 # 512 and 256 columns
 CLASS_LW_FP8 = (512, 512, 256)

@@ -37,7 +37,9 @@ int main() {
   for (int c = 0; c < kNumClasses; ++c) {
     const int lw = class_lw(c), R = class_rows(c), nt = class_nt(c);
     CHECK(lw * R * 2 == 65536);
-    for (int kc = c; kc < kNumClasses; ++kc) CHECK(class_mt(c, consumer_warps_for(kc)) * nt == acc_frags(kc));
+    for (int kc = c; kc < kNumClasses; ++kc) CHECK(class_mt(c, consumer_warps_for(kc)) * nt <= acc_frags(kc));
+    CHECK(acc_frags(c) == (c == 0 ? class_mt(0, 16) * nt : cmax(acc_frags(c - 1), class_mt(c, 16) * nt)));
+    CHECK(acc_frags(c) * 4 <= 32);  // accumulator floats a consumer thread holds
     CHECK(consumer_warps_for(c) == 16);
     CHECK(lw % (consumer_warps_for(c) * 16) == 0);
     CHECK(R % 16 == 0 && R % kBoxRows == 0);
