@@ -121,7 +121,7 @@ __host__ __device__ constexpr int fp8_stage_xoff(int c) { return fp8_stage_wbyte
 constexpr int kFp8XPitch = kFp8Rows * 2 + 16;  // bytes per token row of activations
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
 // Consumer warps: sixteen in every instance (seventeen warps with the
-// producer cap a thread at 96 registers, room for the 32 accumulators).
+// producer cap a thread at 96 registers, room for up to 32 accumulators).
 __host__ __device__ constexpr int consumer_warps_for(int) { return 16; }
 __host__ __device__ constexpr int expert_threads(int kc) { return (consumer_warps_for(kc) + 1) * 32; }
 // m-tiles (16 columns) per consumer warp for class c with cw consumer warps
