@@ -50,11 +50,11 @@
 // Panels.  Each matrix is cut into column panels and K-row stages of 64 KB
 // of weights.  A unit with n tokens takes the panel of its token class, the
 // narrower the more token tiles it has, so that a consumer warp's columns x
-// token tiles -- its accumulators -- stay within 32 fp32 registers:
+// token tiles -- its accumulators -- stay within 64 fp32 registers:
 //   class 0: n <=  8 : 1024 local columns, 32-row stages (1 token tile)
 //   class 1: n <= 16 : 1024 local columns, 32-row stages (2 token tiles)
 //   class 2: n <= 32 :  512 local columns, 64-row stages (4 token tiles)
-// -- 16 consumer warps in every instance, each with 16 (class 0 only) or 32
+// -- 8 consumer warps in every instance, each with 32 (class 0 only) or 64
 // accumulators.  Class 0 is not the wider 2048 x 16 shape its one token tile
 // would allow: a hidden size of 7 x 1024 (7168) cuts into 2048-column DOWN
 // panels with a half-empty last one, and a stage costs about the same ring
@@ -96,8 +96,8 @@ constexpr int kUnitTok = kMaxUnitTokens;  // tokens of one unit, at most
 constexpr int kNumClasses = 3;
 // Token classes.  Every stage holds lw x rows = 32K weights (64 KB): 1024 x
 // 32 for 1-8 tokens (one 8-token tile) and for 9-16 (two tiles), 512 x 64
-// for 17-32 (four tiles); a consumer warp keeps four accumulator fragments
-// (16 floats) in class 0 and eight (32 floats) in classes 1 and 2.
+// for 17-32 (four tiles); a consumer warp keeps eight accumulator fragments
+// (32 floats) in class 0 and sixteen (64 floats) in classes 1 and 2.
 __host__ __device__ constexpr int class_lw(int c) { return c == 2 ? 512 : 1024; }
 __host__ __device__ constexpr int class_rows(int c) { return c == 2 ? 64 : 32; }
 __host__ __device__ constexpr int class_nt(int c) { return c == 0 ? 1 : (c == 1 ? 2 : 4); }
@@ -120,20 +120,29 @@ __host__ __device__ constexpr int fp8_stage_wbytes(int c) { return class_lw_fp8(
 __host__ __device__ constexpr int fp8_stage_xoff(int c) { return fp8_stage_wbytes(c) + 1024; }
 constexpr int kFp8XPitch = kFp8Rows * 2 + 16;  // bytes per token row of activations
 __host__ __device__ constexpr int cmax(int a, int b) { return a > b ? a : b; }
-// Consumer warps: sixteen in every instance (seventeen warps with the
-// producer cap a thread at 96 registers, room for up to 32 accumulators).
-__host__ __device__ constexpr int consumer_warps_for(int) { return 16; }
-__host__ __device__ constexpr int expert_threads(int kc) { return (consumer_warps_for(kc) + 1) * 32; }
+// Consumer warps: eight in the bf16 instances (nine warps with the producer:
+// up to 224 registers a thread, room for 64 accumulators).  Sixteen warps
+// with half the columns each measured slower (batch 1 +0.6 %, batch 8
+// +2.3 %, batch 64 +3.5 %): the extra warps add contention for the stage's
+// shared memory more than they hide its latency; four are slower still.  The
+// e4m3 instances, whose conversions make a stage twice the work, keep
+// sixteen (eight measured 1.5-2 % slower there).
+__host__ __device__ constexpr int consumer_warps_for(int, bool fp8 = false) { return fp8 ? 16 : 8; }
+__host__ __device__ constexpr int expert_threads(int kc, bool fp8 = false) {
+  return (consumer_warps_for(kc, fp8) + 1) * 32;
+}
 // m-tiles (16 columns) per consumer warp for class c with cw consumer warps
 __host__ __device__ constexpr int class_mt(int c, int cw) { return class_lw(c) / (cw * 16); }
 __host__ __device__ constexpr int geo_mt(int c, int cw, bool fp8) { return geo_lw(c, fp8) / (cw * 16); }
 // accumulator fragments (of 4 floats) a consumer thread needs for classes <= KC
-__host__ __device__ constexpr int class_frags(int c, int cw) { return class_mt(c, cw) * class_nt(c); }
-__host__ __device__ constexpr int acc_frags(int kc) {
-  return kc <= 0 ? class_frags(0, consumer_warps_for(kc))
-                 : cmax(acc_frags(kc - 1), class_frags(kc, consumer_warps_for(kc)));
+__host__ __device__ constexpr int class_frags(int c, int cw, bool fp8 = false) {
+  return geo_mt(c, cw, fp8) * class_nt(c);
 }
-static_assert(acc_frags(0) == 4 && acc_frags(1) == 8 && acc_frags(2) == 8, "16 or 32 accumulators a thread");
+__host__ __device__ constexpr int acc_frags(int kc, bool fp8 = false) {
+  return kc <= 0 ? class_frags(0, consumer_warps_for(kc, fp8), fp8)
+                 : cmax(acc_frags(kc - 1, fp8), class_frags(kc, consumer_warps_for(kc, fp8), fp8));
+}
+static_assert(acc_frags(0) == 8 && acc_frags(1) == 16 && acc_frags(2) == 16, "32 or 64 accumulators a thread");
 // stage buffers: weights (row pitch 2*lw + 16 on the plain-copy path) and
 // the tokens' activation rows (pitch 2*rows + 16), largest over the classes
 __host__ __device__ constexpr int stage_w_bytes(int c) { return class_rows(c) * (class_lw(c) * 2 + 16); }
@@ -145,9 +154,8 @@ static_assert(fp8_stage_xoff(0) + 8 * kFp8XPitch <= kStageBytesMma &&
                   fp8_stage_xoff(1) + 16 * kFp8XPitch <= kStageBytesMma &&
                   fp8_stage_xoff(2) + 32 * kFp8XPitch <= kStageBytesMma,
               "fp8 stages: weights, scale row and the class's token rows fit one stage");
-static_assert(geo_mt(0, 16, true) * class_nt(0) <= acc_frags(0) && geo_mt(1, 16, true) * class_nt(1) <= acc_frags(1) &&
-                  geo_mt(2, 16, true) * class_nt(2) <= acc_frags(2),
-              "fp8 classes need no more accumulators than the bf16 instance of the same class");
+static_assert(acc_frags(0, true) == 2 && acc_frags(1, true) == 4 && acc_frags(2, true) == 4,
+              "e4m3 instances: 8 or 16 accumulators a thread");
 constexpr int kMaxStagesMma = 3;
 constexpr int kMaxChunk = 64;  // stages per queue grab, at most
 // tensor-map path: boxes of {64 columns, 16 rows, 4 column chunks}
@@ -1034,7 +1042,7 @@ __device__ __forceinline__ void producer_loop(const MmaArgs& args, const ExpertT
 }
 
 template <int KC, bool TMAP, bool FP8 = false>
-__global__ void __launch_bounds__(expert_threads(KC), 1)
+__global__ void __launch_bounds__(expert_threads(KC, FP8), 1)
     expert_mlp_kernel(const __grid_constant__ MmaArgs args, const __grid_constant__ ExpertTable tab13,
                       const __grid_constant__ ExpertTable tab2) {
   extern __shared__ __align__(1024) uint8_t mma_smem[];
@@ -1046,7 +1054,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   StageHdr* hdr = sv.hdr;
   volatile int* s_misc = sv.s_misc;
 
-  constexpr int CW = consumer_warps_for(KC);
+  constexpr int CW = consumer_warps_for(KC, FP8);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool is_producer = (warp == CW);
 
@@ -1073,7 +1081,7 @@ __global__ void __launch_bounds__(expert_threads(KC), 1)
   } else {
     // =============================================================== consumers
     // (they read nothing the router writes: the stage headers carry it)
-    constexpr int NF = acc_frags(KC);
+    constexpr int NF = acc_frags(KC, FP8);
     float acc[NF][4];
     uint32_t q = 0;
     while (true) {

@@ -468,7 +468,7 @@ int enqueue_forward(moe_decode_ctx* h, const void* x, const void* router_w, cons
   const int n_su = shared_units(s, batch);
   const int kc = kernel_class(batch);
   const MlpKernel mlp = f8 ? pick_mlp_fp8(kc) : (h->use_tc ? moe::expert_tc_kernel : pick_mlp(kc, h->use_tmap));
-  const int mlp_threads = h->use_tc ? moe::kTcThreads : moe::expert_threads(kc);
+  const int mlp_threads = f8 ? moe::expert_threads(kc, true) : (h->use_tc ? moe::kTcThreads : moe::expert_threads(kc));
   const int n_stages = h->use_tc ? h->n_stages_tc : h->n_stages;
   const size_t smem = h->use_tc ? moe::tc_smem_bytes(n_stages) : moe::mma_smem_bytes(n_stages);
 

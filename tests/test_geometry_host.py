@@ -38,9 +38,12 @@ int main() {
     const int lw = class_lw(c), R = class_rows(c), nt = class_nt(c);
     CHECK(lw * R * 2 == 65536);
     for (int kc = c; kc < kNumClasses; ++kc) CHECK(class_mt(c, consumer_warps_for(kc)) * nt <= acc_frags(kc));
-    CHECK(acc_frags(c) == (c == 0 ? class_mt(0, 16) * nt : cmax(acc_frags(c - 1), class_mt(c, 16) * nt)));
-    CHECK(acc_frags(c) * 4 <= 32);  // accumulator floats a consumer thread holds
-    CHECK(consumer_warps_for(c) == 16);
+    const int cw = consumer_warps_for(c);
+    CHECK(acc_frags(c) == (c == 0 ? class_mt(0, cw) * nt : cmax(acc_frags(c - 1), class_mt(c, cw) * nt)));
+    CHECK(acc_frags(c) * 4 <= 64);  // accumulator floats a consumer thread holds
+    CHECK(cw == 8 && expert_threads(c) == 288);
+    CHECK(consumer_warps_for(c, true) == 16 && expert_threads(c, true) == 544);
+    for (int kc = c; kc < kNumClasses; ++kc) CHECK(class_frags(c, consumer_warps_for(kc, true), true) <= acc_frags(kc, true));
     CHECK(lw % (consumer_warps_for(c) * 16) == 0);
     CHECK(R % 16 == 0 && R % kBoxRows == 0);
     CHECK((lw / 2) % (kChunkCols * kBoxChunks) == 0);
