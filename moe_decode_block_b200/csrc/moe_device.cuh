@@ -191,11 +191,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int c0, 
       : "memory");
 }
 
-// Bulk prefetch of a global range into L2 (no data returned to the SM).
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // Fire-and-forget fp32 adds to global memory (no value comes back, so a warp
 // issuing many of them never waits on their round trips).  Vector forms need
 // the address aligned to the vector size.
