@@ -69,6 +69,9 @@ def parse_args():
     p.add_argument("--no-configs", action="store_true", help="skip the other graded configurations")
     p.add_argument("--config-steps", type=int, default=200, help="timed graph replays per extra configuration")
     p.add_argument("--no-parity", action="store_true", help="skip the oracle check of the timed forwards")
+    p.add_argument("--chain", type=int, default=0,
+                   help="measure a chain of this many blocks of the config (one handle per block, distinct "
+                        "weights) against its first block alone: graph replays, L2 flushed; prints that line")
     p.add_argument("--fp8-forwards", type=int, default=0,
                    help="profiling driver: run this many e4m3-weight forwards of the config (L2 flushed before "
                         "each), print their event-timed us and exit (no bench line)")
@@ -451,6 +454,8 @@ def run_ours(args):
     if args.fp8_forwards > 0:
         fp8_forwards(wl, args.fp8_forwards, args.seed, dev)
         return
+    if args.chain > 0:
+        return chain_bench(wl, args.chain, args.seed, dev, args.steps, args.warmup)
     wts, x, margin = make_inputs(wl, args.seed, args.seed + 1000 * rank, dev)
     main = torch.cuda.Stream()
     aux = torch.cuda.Stream()
@@ -771,6 +776,80 @@ def fp8_forwards(wl, n, seed, dev):
     print(json.dumps({"fp8_forwards": wl.name, "us": us, "device_status": status}), flush=True)
     if status != 0:
         raise SystemExit(f"device status {status}")
+
+
+def chain_bench(wl, n_blocks, seed, dev, steps, warmup):
+    """A chain of n_blocks blocks of the workload (block 0 on the config's
+    weights and input, block l on the weights of seed + l) timed as one CUDA
+    graph per step, against a graph of block 0 alone; L2 flushed before every
+    replay.  Prints one JSON line; returns non-zero on a device error."""
+    import numpy as np
+    import torch
+    from moe_decode_block_b200 import synth
+    from moe_decode_block_b200.chain import BlockChain
+    s, B = wl.shape, wl.batch
+    wts0, x, _ = make_inputs(wl, seed, seed, dev)
+    weights = [wts0] + [synth.make_weights(s, seed=seed + l, device=dev, routing=wl.routing)
+                        for l in range(1, n_blocks)]
+    chain = BlockChain(n_blocks, s.hidden, s.n_experts, s.top_k, s.inter, s.shared_inter, n_shared=s.n_shared,
+                       max_batch=max(B, 1), router_biases=[w.router_bias for w in weights])
+    outs = [torch.empty_like(x) for _ in range(n_blocks)]
+    ids = [torch.empty(B, s.top_k, dtype=torch.int32, device=dev) for _ in range(n_blocks)]
+    ws = [torch.empty(B, s.top_k, dtype=torch.float32, device=dev) for _ in range(n_blocks)]
+    wl_args = [(w.router_w, w.w13, w.w2, w.shared_w13, w.shared_w2) for w in weights]
+    main_s = torch.cuda.Stream()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    fb = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    fs = torch.empty((), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(main_s):
+        chain.forward(x, wl_args, outs, ids, ws, stream=main_s)
+    main_s.synchronize()
+    if chain.status() != 0:
+        chain.close()
+        raise SystemExit(f"device status {chain.status()} after the first chain forward")
+    bytes_blocks = [bytes_per_step(s, ids[l].cpu().numpy(), B)[0] for l in range(n_blocks)]
+    g_chain, g_one = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_chain, stream=main_s):
+        chain.forward(x, wl_args, outs, ids, ws, stream=torch.cuda.current_stream())
+    with torch.cuda.graph(g_one, stream=main_s):
+        chain.blocks[0].forward(x, *wl_args[0], outs[0], ids[0], ws[0], stream_main=torch.cuda.current_stream())
+
+    def timed(g):
+        with torch.cuda.stream(main_s):
+            for _ in range(warmup):
+                fb.zero_()
+                torch.sum(fb, dim=0, out=fs)
+                g.replay()
+        torch.cuda.synchronize()
+        sampler = ClockSampler(dev.index)
+        sampler.start()
+        time.sleep(0.2)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        with torch.cuda.stream(main_s):
+            for a, b in ev:
+                fb.zero_()
+                torch.sum(fb, dim=0, out=fs)
+                a.record(main_s)
+                g.replay()
+                b.record(main_s)
+        torch.cuda.synchronize()
+        return float(np.median([a.elapsed_time(b) for a, b in ev])) * 1e3, sampler.stop()
+
+    us_one, clocks_one = timed(g_one)
+    us_chain, clocks_chain = timed(g_chain)
+    status = chain.status()
+    del g_chain, g_one
+    chain.close()
+    line = {"chain": {"workload": wl.name, "blocks": n_blocks, "batch": B, "steps": steps, "warmup": warmup,
+                      "us_block_alone": round(us_one, 2), "us_chain": round(us_chain, 2),
+                      "us_per_block_in_chain": round(us_chain / n_blocks, 2),
+                      "GB/s_chain": round(sum(bytes_blocks) / (us_chain * 1e-6) / 1e9, 1),
+                      "GB/s_block_alone": round(bytes_blocks[0] / (us_one * 1e-6) / 1e9, 1),
+                      "l2": "flushed before every replay (of the chain, or of the block alone)",
+                      "clocks_block_alone": clocks_one, "clocks_chain": clocks_chain,
+                      "device_status": status}}
+    print(json.dumps(line), flush=True)
+    return 0 if status == 0 else 1
 
 
 def main():
