@@ -63,7 +63,7 @@ def _run_chain(shape, n_blocks, B, seed0, max_batch=64):
         for l in range(n_blocks):
             xin = x if l == 0 else outs[l - 1]
             compared += chain_block_check(weights[l], shape.top_k, xin, outs[l], ids[l], ws[l])
-        assert compared >= n_blocks * B - 1  # near-ties are rare
+        assert compared >= n_blocks * B - max(1, n_blocks * B // 20)  # near-ties are rare
     finally:
         chain.close()
 
